@@ -1,0 +1,449 @@
+"""Benchmark of the block-sparse FlashAttention forward on B200.
+
+Headline workload (one step = one pass of the hot path over one batch):
+speculative + sparse decode, B=8, Hq=32, Hkv=8 (GQA 4), Lq=1, Lk=32768,
+D=128, bf16, block 128: dense over the last 2048 keys plus 32 random missed
+blocks per (b, kv-head), merged by the LSE combine -- one fused split-KV
+kernel launch.  Metric: kept-K/V GB/s (algorithmic bytes: the distinct K and
+V bytes attended + q + o + lse + table) against the measured HBM copy
+bandwidth.
+
+The prefill workloads (tiny block table, gated BSFA prefill at 32K,
+vertical-slash prefill at 128K) are timed in the same run and reported under
+"prefill" with kept-block TFLOP/s against the measured bf16 tensor peak.
+
+python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Under torchrun each rank runs its own replica (independent problems, no
+data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = ("sparse-attn fwd kept-block TFLOP/s (% bf16 peak); "
+          "decode kept-KV GB/s (% HBM)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CSRC = os.path.join(ROOT, "block_sparse_flashattention_sbfa_b200", "csrc")
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def source_sha():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        h.update(open(os.path.join(CSRC, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    if not e or e.get("source_sha") != source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap,utilization.gpu")
+
+    def __init__(self, gpu):
+        self.gpu = gpu
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        loaded = [s for s in self.samples if s[6].isdigit() and int(s[6]) > 0] or self.samples
+        sm = [int(s[0]) for s in loaded if s[0].isdigit()]
+        reasons = sorted({names[i] for s in loaded for i in range(4) if s[2 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": int(self.samples[0][1]) if self.samples[0][1].isdigit() else None,
+                "reasons": reasons, "samples": len(loaded)}
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, torch):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self, torch):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, torch, x):
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def time_device(torch, dist, fn, steps, warmup, flush):
+    """Per-step CUDA-event time of fn (ms, mean over steps; max over ranks).
+    The L2 flush runs between steps outside the events."""
+    for _ in range(warmup):
+        fn()
+        flush()
+    dist.barrier(torch)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    t0 = time.perf_counter()
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+        flush()
+    torch.cuda.synchronize()
+    dist.barrier(torch)
+    wall = time.perf_counter() - t0
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    return dist.max(torch, ms), wall
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def decode_bytes(wl):
+    t = wl.meta["table"]
+    B, Lk, Hkv, D = wl.k.shape
+    Hq = wl.q.shape[2]
+    bs = wl.meta["kv_block"]
+    spec = wl.meta["spec_end"] - wl.meta["spec_begin"]
+    keys = 0
+    for b in range(B):
+        for g in range(Hkv):
+            blocks = set(int(x) for x in t[b, g, 0] if x >= 0)
+            keys += spec + sum(min(bs, Lk - j * bs) for j in blocks)
+    kv = keys * D * 2 * 2
+    qo = 2 * B * wl.q.shape[1] * Hq * D * 2 + B * Hq * wl.q.shape[1] * 4 + t.size * 4
+    return kv + qo, kv
+
+
+def bench_decode(torch, sb, dist, args, flush, peaks):
+    wl = W.make_spec_decode()
+    s0 = wl.meta["spec_begin"]
+    q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
+    tab = torch.from_numpy(wl.meta["table"]).cuda()
+    ws = sb.decode_workspace(8, 8, 1, 32, "cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty(8, 32, 1, dtype=torch.float32, device="cuda")
+    ks, vs = k[:, s0:], v[:, s0:]
+
+    def step():
+        sb.speculative_sparse(q, ks, vs, True, k, v, tab, 128, ws=ws, out=o, lse=lse)
+
+    ms, wall = time_device(torch, dist, step, args.steps, args.warmup, flush)
+    nbytes, kv = decode_bytes(wl)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res = dict(ms=ms, gbs=gbs, bytes=nbytes, kv_bytes=kv, wall=wall)
+    # end to end through the public API: host buffers in, result back out
+    hq, hk, hv = (W.to_torch_bf16(x).pin_memory() for x in (wl.q, wl.k, wl.v))
+    ht = torch.from_numpy(wl.meta["table"]).pin_memory()
+    ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        tab.copy_(ht, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    ems, _ = time_device(torch, dist, e2e_step, e2e_steps, 1, lambda: None)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ht))
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    res["e2e"] = {"value": round(nbytes / (ems * 1e-3) / 1e9, 3), "unit": "GB/s",
+                  "ms_per_step": round(ems, 4), "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h,
+                  "note": "host->device copy of q, k, v (the whole cache) and table every step"}
+    res["wl"] = wl
+    return res
+
+
+def gated_flops(keep, L, Hq, block=64):
+    n = keep.shape[-1]
+    n_qk = Hq * L * (L + 1) // 2
+    diag = block * (block + 1) // 2
+    n_pv = 0
+    for h in range(Hq):
+        kh = keep[0, h]
+        tri = np.tril(kh.astype(np.int64), -1).sum()
+        n_pv += int(tri) * block * block + n * diag
+    return 2 * 128 * n_qk + 2 * 128 * n_pv, n_qk, n_pv
+
+
+def bench_gated(torch, sb, dist, args, flush, peaks):
+    T = np.load(os.path.join(ROOT, "tests", "golden", "gated_T_seed101.npy"))
+    wl = W.make_gated()
+    q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
+    Tg = torch.from_numpy(T).cuda()
+    n = T.shape[1]
+    keep = torch.zeros((1, 32, n, n), dtype=torch.uint8, device="cuda")
+    o, lse = sb.fwd_gated(q, k, v, Tg, keep_out=keep)
+    torch.cuda.synchronize()
+    flops, n_qk, n_pv = gated_flops(keep.cpu().numpy(), 32768, 32)
+    kept = int(keep.sum().item())
+    ms, _ = time_device(torch, dist, lambda: sb.fwd_gated(q, k, v, Tg, out=o, lse=lse),
+                        max(3, args.steps // 10), args.warmup, flush)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": "gated BSFA prefill B=1 Hq=32 Hkv=8 L=32768 causal D=128 bf16 64x64 "
+                        "tiles, T from seed-101 calibration (k=64)",
+            "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
+            "kept_tile_density": round(kept / (32 * n * (n + 1) / 2), 4),
+            "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+
+
+def vs_flops(bc, bo, cc, ci, L, block=64):
+    B, H, nqb = bc.shape
+    diag = block * (block + 1) // 2
+    pairs = 0
+    for h in range(H):
+        for i in range(nqb):
+            offs = bo[0, h, i, :bc[0, h, i]] // block
+            pairs += int((offs < i).sum()) * block * block + int((offs == i).sum()) * diag
+            cols = ci[0, h, i, :cc[0, h, i]].astype(np.int64)
+            m0, m1 = i * block, min((i + 1) * block, L)
+            pairs += int(np.minimum(block, np.maximum(m1 - np.maximum(cols, m0), 0)).sum())
+    return 4 * 128 * pairs, pairs
+
+
+def bench_vs(torch, sb, dist, args, flush, peaks):
+    wl = W.make_vertical_slash()
+    L = wl.q.shape[1]
+    q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    vt = torch.from_numpy(wl.meta["vertical"]).cuda()
+    st = torch.from_numpy(wl.meta["slash"]).cuda()
+    conv = lambda: sb.convert_vertical_slash(sl, sl, vt, st, L)  # noqa: E731
+    bc, bo, cc, ci = conv()
+    o, lse = sb.fwd_vertical_slash(q, k, v, bc, bo, cc, ci, causal=True)
+    torch.cuda.synchronize()
+    flops, pairs = vs_flops(bc.cpu().numpy(), bo.cpu().numpy(), cc.cpu().numpy(),
+                            ci.cpu().numpy(), L)
+    steps = max(3, args.steps // 50)
+    ms, _ = time_device(torch, dist, lambda: sb.fwd_vertical_slash(
+        q, k, v, bc, bo, cc, ci, causal=True, out=o, lse=lse), steps, min(args.warmup, 3), flush)
+    cms, _ = time_device(torch, dist, conv, steps, 1, flush)
+    tf = flops / (ms * 1e-3) / 1e12
+    dense = 4 * 128 * 32 * L * (L + 1) // 2
+    return {"workload": "vertical-slash prefill B=1 H=32 L=131072 causal D=128 bf16 "
+                        "BM=BN=64, 1000 vertical + 6000 slash per head",
+            "ms": round(ms, 3), "tflops": round(tf, 2), "flops": flops,
+            "frac_of_causal_dense": round(flops / dense, 4),
+            "convert_ms": round(cms, 4),
+            "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+
+
+def bench_table(torch, sb, dist, args, flush, peaks):
+    wl = W.make_block_table()
+    q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
+    t = torch.from_numpy(wl.meta["table"]).cuda()
+    o, lse = sb.fwd(q, k, v, t, 64, 64)
+    ms, _ = time_device(torch, dist, lambda: sb.fwd(q, k, v, t, 64, 64, out=o, lse=lse),
+                        args.steps, args.warmup, flush)
+    flops = 4 * 128 * 2 * 256 * 8 * 64
+    return {"workload": "block table B=1 H=2 Lq=256 Lk=1024 bs=64 (diag + 7 random of 16)",
+            "ms": round(ms, 5), "tflops": round(flops / (ms * 1e-3) / 1e12, 3),
+            "note": "launch-bound correctness workload"}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def cpu_baseline_decode(wl, budget_s=15.0):
+    import oracle
+    t = wl.meta["table"]
+    s0 = wl.meta["spec_begin"]
+    nbytes, _ = decode_bytes(wl)
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        oracle.speculative_sparse(wl.q, wl.k[:, s0:], wl.v[:, s0:], True, wl.k, wl.v, t, 128,
+                                  wl.scale)
+        done += 1
+        if time.perf_counter() - t0 > budget_s or done >= 3:
+            break
+    sec = (time.perf_counter() - t0) / done
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((x.get("num_threads", 1) for x in threadpool_info()), default=1)
+    except Exception:
+        blas = None
+    return {"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": os.cpu_count(),
+            "blas_threads": blas, "kind": "oracle",
+            "sample": f"the whole decode workload (all 256 (b, h) rows), {done} pass(es), "
+                      f"{sec:.2f} s per pass"}
+
+
+# ----------------------------------------------------------------------------
+# main
+# ----------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--headline-only", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    dist = Dist()
+    peaks, peak_kind = load_peaks()
+
+    if args.impl == "reference":
+        if dist.rank != 0:
+            return
+        wl = W.make_spec_decode()
+        cb = cpu_baseline_decode(wl, budget_s=20.0)
+        sec_per_step = decode_bytes(wl)[0] / (cb["value"] * 1e9)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(sec_per_step * 1e3, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "speculative+sparse decode B=8 Hq=32 Hkv=8 Lq=1 "
+                                       "Lk=32768 D=128 bs=128, dense last 2048 + 32 missed "
+                                       "blocks", "global_batch": 8, "seq_len": 32768},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    torch.cuda.set_device(dist.local)
+    dist.init(torch)
+    import block_sparse_flashattention_sbfa_b200 as sb
+
+    l2 = torch.cuda.get_device_properties(dist.local).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.fill_(1)  # noqa: E731
+
+    clocks = ClockSampler(dist.local).start()
+    dec = bench_decode(torch, sb, dist, args, flush, peaks)
+    prefill = {}
+    if not args.headline_only:
+        for name, fn in (("gated", bench_gated), ("vertical_slash", bench_vs),
+                         ("block_table", bench_table)):
+            try:
+                prefill[name] = fn(torch, sb, dist, args, flush, peaks)
+            except Exception as e:  # report, keep the headline
+                prefill[name] = {"error": f"{type(e).__name__}: {e}"}
+    ck = clocks.stop()
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1:
+        cpu = cpu_baseline_decode(dec["wl"])
+    value = dec["gbs"] * dist.world
+    achieved = dec["bytes"] / (dec["ms"] * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dec["ms"], 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "speculative+sparse decode B=8 Hq=32 Hkv=8 Lq=1 Lk=32768 "
+                               "D=128 bs=128, dense last 2048 + 32 missed blocks, fused "
+                               "split-KV kernel", "global_batch": 8 * dist.world,
+                   "seq_len": 32768, "parallelism": f"replicas x{dist.world}",
+                   "l2": "flushed between steps (2x L2 write), outside the timed events"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic("decode_kernel"), "peak_kind": peak_kind,
+                     "kernel": "decode_kernel", "algorithmic_bytes": dec["bytes"]},
+        "e2e": dec["e2e"],
+        "gpu_launches": args.steps,
+        "clocks": ck,
+        "prefill": prefill,
+    }
+    if cpu:
+        line["cpu_baseline"] = cpu
+    if dist.rank == 0:
+        print(json.dumps(line))
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,122 @@
+// Vertical/slash index conversion (Sglang Sparse Flash Attention,
+// convert_vertical_slash_indexes): one CTA per (batch, head, q-block).
+//
+// Slash offset s is the diagonal key = row + d - s (d = kv_len - q_len); over
+// the q-block's rows [m0, m1) it covers keys [m0+d-s, m1-1+d-s].  Each such
+// range is at most 64 keys long, so it touches at most two 64-key blocks; the
+// CTA marks them in a shared bitmap, then compacts the bitmap into the
+// ascending block_offset list.  Vertical columns that are visible and not
+// inside a listed block are compacted, in order, into column_index.
+#pragma once
+
+#include "sbfa_ptx.cuh"
+
+namespace sbfa {
+
+constexpr int kCvThreads = 128;
+constexpr int kCvMaxWords = 8192 / 32;  // kv_len <= 524288 (64-key blocks)
+
+// Exclusive block-wide prefix sum over kCvThreads values; returns the total.
+__device__ __forceinline__ int cv_block_scan(int v, int* warp_tot, int& excl) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  int base = 0, total = 0;
+  for (int w = 0; w < kCvThreads / 32; ++w) {
+    if (w < warp) base += warp_tot[w];
+    total += warp_tot[w];
+  }
+  excl = base + x - v;
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kCvThreads)
+    convert_vs_kernel(const int* __restrict__ q_seqlens, const int* __restrict__ kv_seqlens,
+                      const int* __restrict__ vertical, int nnz_v, const int* __restrict__ slash,
+                      int nnz_s, int H, int nqb, int block_M, int block_N, int causal,
+                      int* __restrict__ block_count, int* __restrict__ block_offset,
+                      int* __restrict__ column_count, int* __restrict__ column_index,
+                      int* status) {
+  __shared__ uint32_t bm[kCvMaxWords];
+  __shared__ int warp_tot[kCvThreads / 32];
+  const int i = blockIdx.x % nqb;
+  const int bh = blockIdx.x / nqb;
+  const int b = bh / H;
+  const int tid = threadIdx.x;
+  const int q_len = q_seqlens[b], kv_len = kv_seqlens[b];
+  const int d = kv_len - q_len;
+  const int64_t row = static_cast<int64_t>(bh) * nqb + i;
+  const int m0 = i * block_M;
+  if (m0 >= q_len) {
+    if (tid == 0) {
+      block_count[row] = 0;
+      column_count[row] = 0;
+    }
+    return;
+  }
+  const int m1 = min(m0 + block_M, q_len);
+  const int nkb = (kv_len + block_N - 1) / block_N;
+  const int nwords = (nkb + 31) >> 5;
+  for (int w = tid; w < nwords; w += kCvThreads) bm[w] = 0u;
+  __syncthreads();
+  const int* sl = slash + static_cast<int64_t>(bh) * nnz_s;
+  for (int e = tid; e < nnz_s; e += kCvThreads) {
+    const int s = sl[e];
+    if (s < 0) { report(status, kDevBadIndex); continue; }
+    const int lo = max(m0 + d - s, 0);
+    const int hi = min(m1 - 1 + d - s, kv_len - 1);
+    if (hi < lo) continue;
+    for (int j = lo / block_N; j <= hi / block_N; ++j) atomicOr(&bm[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  // ---- compact the bitmap into ascending block offsets
+  int* bo = block_offset + row * nnz_s;
+  int written = 0;
+  for (int w0 = 0; w0 < nwords; w0 += kCvThreads) {
+    const int w = w0 + tid;
+    const uint32_t bits = w < nwords ? bm[w] : 0u;
+    int excl;
+    const int tot = cv_block_scan(__popc(bits), warp_tot, excl);
+    int pos = written + excl;
+    uint32_t x = bits;
+    while (x) {
+      const int bit = __ffs(x) - 1;
+      x &= x - 1u;
+      if (pos < nnz_s) bo[pos] = (w * 32 + bit) * block_N;
+      ++pos;
+    }
+    written += tot;
+  }
+  if (tid == 0) {
+    if (written > nnz_s) report(status, kDevOverflow);
+    block_count[row] = min(written, nnz_s);
+  }
+  // ---- vertical columns not covered by a listed block
+  const int* vt = vertical + static_cast<int64_t>(bh) * nnz_v;
+  int* ci = column_index + row * nnz_v;
+  const int vis_end = causal ? min(kv_len, m1 + d) : kv_len;  // columns < vis_end
+  int ncol = 0;
+  for (int e0 = 0; e0 < nnz_v; e0 += kCvThreads) {
+    const int e = e0 + tid;
+    int c = -1;
+    bool keep = false;
+    if (e < nnz_v) {
+      c = vt[e];
+      keep = c >= 0 && c < vis_end && !((bm[(c / block_N) >> 5] >> ((c / block_N) & 31)) & 1u);
+      if (c < 0) report(status, kDevBadIndex);
+    }
+    int excl;
+    const int tot = cv_block_scan(keep ? 1 : 0, warp_tot, excl);
+    if (keep) ci[ncol + excl] = c;
+    ncol += tot;
+  }
+  if (tid == 0) column_count[row] = ncol;
+}
+
+}  // namespace sbfa

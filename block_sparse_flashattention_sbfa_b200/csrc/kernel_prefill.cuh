@@ -1,0 +1,774 @@
+// Block-sparse FlashAttention forward on the 5th-generation tensor cores.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer for Q and K tiles; builds each work unit's
+//               key-tile schedule in shared memory
+//   warp 1      tcgen05 MMA issuer (one elected lane); owns the TMEM allocation
+//   warp 2      producer for V tiles (waits for the gate's keep decision in
+//               gated mode: pruned blocks load no V, BSFA Figure 2b) and for
+//               gathered vertical columns
+//   warp 3      gathers K rows of vertical columns
+//   warps 4-7   softmax warpgroup of Q tile 0 (one thread per query row)
+//   warps 8-11  softmax warpgroup of Q tile 1
+//
+// Work unit: four 64-row "segments" (head, query rows) that share one kv head:
+// with GQA they are heads of one group at the same q-block (K/V tiles are
+// loaded once for all of them); without GQA they are four consecutive
+// q-blocks of one head.  Segments 0,1 form M = 128 tile 0 and segments 2,3
+// tile 1.  Each segment has a set of 64-key tiles (from the block table, the
+// causal range, the gate candidates or the vertical/slash lists); the unit
+// walks the union of the four sets in ascending order and runs
+//   S_t = Q_t K^T  (tcgen05.mma, M128 N64 K128, fp32 in TMEM)
+//   softmax rows, P_t (bf16) -> shared memory
+//   O_t += P_t V   (tcgen05.mma, M128 N128 K64, fp32 in TMEM)
+// for every tile t with an active segment; rows of an inactive segment get
+// P = 0.  The online softmax keeps a lazily updated running max (rescale O
+// only when the max grows by more than 2^8), which leaves o and lse exact.
+//
+// TMEM (512 columns): tile t uses columns [256t, 256t+256): S buffers 0/1 at
+// +0/+64 (64 fp32 columns each), O at +128 (128 columns).
+#pragma once
+
+#include "sbfa_ptx.cuh"
+
+namespace sbfa {
+
+enum PrefillMode : int { kModeTable = 0, kModeDense = 1, kModeGated = 2, kModeVS = 3 };
+
+constexpr int kPfThreads = 384;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr int kMaxKT = 8192;              // 64-key tiles: Sk <= 524288
+constexpr int kBmWords = kMaxKT / 32;
+constexpr int kDecRingSlots = 4;
+constexpr int kMaxCols = 1024;            // union of vertical columns per unit
+constexpr int kTileBytes = 64 * 128 * 2;  // 64 keys x 128 dims bf16
+constexpr int kQTileBytes = 128 * 128 * 2;
+constexpr int kPTileBytes = 128 * 64 * 2;
+
+struct PrefillParams {
+  int mode;
+  int B, Sq, Sk, Hq, Hkv, G;
+  int hp, subs_per_unit, n_sub, n_hgrp, n_subgrp, n_units, n_kt;
+  int causal, causal_off;
+  float scale, scale_log2;
+  void* o;
+  int64_t osb, oss, osh;
+  int o_f32;
+  float* lse;
+  // table mode
+  const int* idx;
+  int64_t tsb, tsh, tsqb;
+  int nmax, q_block, kv_block, n_kb;
+  // gated mode
+  const float* T;
+  int nqb;
+  float* smax_out;
+  uint8_t* keep_out;
+  // vertical-slash mode
+  const int* vs_bc;
+  const int* vs_bo;
+  int nnz_s;
+  const int* vs_cc;
+  const int* vs_ci;
+  int nnz_v;
+  int vs_nqb;
+  // q/k/v for column gathers
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  int64_t ksb, kss, ksh, vsb, vss, vsh;
+  int* status;
+};
+
+struct PfSched {
+  uint32_t bm[4][kBmWords];
+  int col[kMaxCols];
+  uint8_t colmask[kMaxCols];
+  int n_words, n_cols;
+  int b, g;
+  int seg_valid[4], seg_head[4], seg_row0[4], seg_qb[4];
+  float seg_T[4];
+};
+
+struct PfSmem {
+  alignas(1024) uint8_t q[2][kQTileBytes];
+  alignas(1024) uint8_t k[kKStages][kTileBytes];
+  alignas(1024) uint8_t v[kVStages][kTileBytes];
+  alignas(1024) uint8_t p[2][kPTileBytes];
+  PfSched sched[2];
+  float red[2][2][4];
+  int dec_val[kDecRingSlots][2];
+  int pv_flag[2][2];
+  uint32_t tmem_base;
+  int abort_flag;
+  uint64_t sched_full[2], sched_empty[2];
+  uint64_t q_full[2], q_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2][2], s_empty[2][2];
+  uint64_t p_full[2][2], pv_done[2], o_free[2];
+  uint64_t dec_full[kDecRingSlots], dec_empty[kDecRingSlots];
+};
+
+// Visit the union of the four segments' tile sets in ascending order, then the
+// vertical-column chunks.  fn(item, kt_or_chunk, is_col, mem) with mem = bit s
+// set when segment s takes part; stops early when fn returns false.
+template <class F>
+__device__ __forceinline__ bool pf_for_each(const PfSched& sc, F&& fn) {
+  int item = 0;
+  for (int w = 0; w < sc.n_words; ++w) {
+    const uint32_t b0 = sc.bm[0][w], b1 = sc.bm[1][w], b2 = sc.bm[2][w], b3 = sc.bm[3][w];
+    uint32_t any = b0 | b1 | b2 | b3;
+    while (any) {
+      const int bit = __ffs(any) - 1;
+      any &= any - 1u;
+      const int mem = ((b0 >> bit) & 1) | (((b1 >> bit) & 1) << 1) | (((b2 >> bit) & 1) << 2) |
+                      (((b3 >> bit) & 1) << 3);
+      if (!fn(item++, w * 32 + bit, false, mem)) return false;
+    }
+  }
+  const int nch = (sc.n_cols + 63) >> 6;
+  for (int c = 0; c < nch; ++c) {
+    int mem = 0;
+    const int e1 = min(sc.n_cols, c * 64 + 64);
+    for (int e = c * 64; e < e1; ++e) mem |= sc.colmask[e];
+    if (!fn(item++, c, true, mem)) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void pf_set_range(uint32_t* bm, int t0, int t1) {
+  for (int t = t0; t < t1; ++t) atomicOr(&bm[t >> 5], 1u << (t & 31));
+}
+
+// Build the schedule of unit u (whole warp 0).
+__device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int lane) {
+  const int per_sg = p.B * p.Hkv * p.n_hgrp;
+  const int sg = p.n_subgrp - 1 - u / per_sg;  // heaviest (latest rows) first
+  const int rest = u % per_sg;
+  const int hgrp = rest % p.n_hgrp;
+  const int bg = rest / p.n_hgrp;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  const int n_words = (p.n_kt + 31) >> 5;
+  for (int e = lane; e < 4 * kBmWords; e += 32) (&sc.bm[0][0])[e] = 0u;
+  if (lane == 0) {
+    sc.n_words = n_words;
+    sc.n_cols = 0;
+    sc.b = b;
+    sc.g = g;
+  }
+  __syncwarp();
+  for (int s = 0; s < 4; ++s) {
+    const int hs = s % p.hp, ss = s / p.hp;
+    const int head = g * p.G + hgrp * p.hp + hs;
+    const int sub = sg * p.subs_per_unit + ss;
+    const int valid = sub < p.n_sub;
+    const int row0 = sub * 64;
+    if (lane == 0) {
+      sc.seg_valid[s] = valid;
+      sc.seg_head[s] = head;
+      sc.seg_row0[s] = row0;
+      sc.seg_qb[s] = sub;
+      sc.seg_T[s] = (p.mode == kModeGated && valid) ? p.T[head * p.nqb + sub] : 0.f;
+    }
+    if (!valid) continue;
+    // causal limit: last tile any row of the segment may see
+    int kt_end = p.n_kt;
+    if (p.causal) {
+      const int last_row = min(row0 + 63, p.Sq - 1);
+      const int max_key = last_row + p.causal_off;
+      kt_end = max_key < 0 ? 0 : min(p.n_kt, max_key / 64 + 1);
+    }
+    uint32_t* bm = sc.bm[s];
+    if (p.mode == kModeDense || p.mode == kModeGated) {
+      for (int w = lane; w * 32 < kt_end; w += 32) {
+        const int t0 = w * 32, t1 = min(kt_end, t0 + 32);
+        bm[w] = (t1 - t0 == 32) ? 0xffffffffu : ((1u << (t1 - t0)) - 1u);
+      }
+    } else if (p.mode == kModeTable) {
+      const int qb = row0 / p.q_block;
+      const int* row = p.idx + b * p.tsb + g * p.tsh + qb * p.tsqb;
+      const int tpb = p.kv_block / 64;
+      for (int n = lane; n < p.nmax; n += 32) {
+        const int j = row[n];
+        if (j < 0) continue;
+        if (j >= p.n_kb) { report(p.status, kDevBadIndex); continue; }
+        pf_set_range(bm, j * tpb, min(kt_end, j * tpb + tpb));
+      }
+    } else {  // vertical-slash: listed blocks
+      const int64_t base = (static_cast<int64_t>(b) * p.Hq + head) * p.vs_nqb + sub;
+      const int cnt = min(p.vs_bc[base], p.nnz_s);
+      const int* offs = p.vs_bo + base * p.nnz_s;
+      for (int n = lane; n < cnt; n += 32) {
+        const int off = offs[n];
+        if (off < 0 || off >= p.Sk || (off & 63)) { report(p.status, kDevBadIndex); continue; }
+        const int t = off >> 6;
+        if (t < kt_end) atomicOr(&bm[t >> 5], 1u << (t & 31));
+      }
+    }
+  }
+  __syncwarp();
+  if (p.mode == kModeVS && lane == 0) {
+    // merge the four ascending column lists (union, with segment membership)
+    int cur[4], cnt[4];
+    const int* lst[4];
+    for (int s = 0; s < 4; ++s) {
+      cur[s] = 0;
+      cnt[s] = 0;
+      lst[s] = nullptr;
+      if (!sc.seg_valid[s]) continue;
+      const int64_t base =
+          (static_cast<int64_t>(b) * p.Hq + sc.seg_head[s]) * p.vs_nqb + sc.seg_qb[s];
+      cnt[s] = min(p.vs_cc[base], p.nnz_v);
+      lst[s] = p.vs_ci + base * p.nnz_v;
+    }
+    int n = 0;
+    while (true) {
+      int best = 0x7fffffff;
+      for (int s = 0; s < 4; ++s)
+        if (cur[s] < cnt[s]) best = min(best, lst[s][cur[s]]);
+      if (best == 0x7fffffff) break;
+      int mem = 0;
+      for (int s = 0; s < 4; ++s)
+        if (cur[s] < cnt[s] && lst[s][cur[s]] == best) { mem |= 1 << s; ++cur[s]; }
+      if (best < 0 || best >= p.Sk) { report(p.status, kDevBadIndex); continue; }
+      if (n == kMaxCols) { report(p.status, kDevOverflow); break; }
+      sc.col[n] = best;
+      sc.colmask[n] = static_cast<uint8_t>(mem);
+      ++n;
+    }
+    sc.n_cols = n;
+  }
+  __syncwarp();
+}
+
+// Gather 64 K or V rows (vertical columns of chunk c) into a swizzled tile;
+// rows past the list end are zero-filled.  Whole warp; completes the
+// copies and the proxy fence before returning.
+__device__ __forceinline__ void pf_gather_rows(const PfSched& sc, int c, const __nv_bfloat16* base,
+                                               int64_t sb, int64_t ss, int64_t sh, uint8_t* dst,
+                                               int lane) {
+  const uint32_t d0 = smem_u32(dst);
+  for (int e = lane; e < 64 * 16; e += 32) {
+    const int r = e >> 4, ch = e & 15;  // row, 16-byte chunk of the 256-byte row
+    const int half = ch >> 3, cc = ch & 7;
+    const uint32_t saddr = d0 + half * 8192 + sw128_off(r, cc);
+    const int idx = c * 64 + r;
+    if (idx < sc.n_cols) {
+      const __nv_bfloat16* src = base + sc.b * sb + static_cast<int64_t>(sc.col[idx]) * ss +
+                                 sc.g * sh + ch * 8;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(src) : "memory");
+    } else {
+      asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(saddr), "r"(0) : "memory");
+    }
+  }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
+                   const __grid_constant__ CUtensorMap mapK,
+                   const __grid_constant__ CUtensorMap mapV, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  PfSmem& sm = *reinterpret_cast<PfSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.sched_full[i], 1);
+      mbar_init(&sm.sched_empty[i], 1 + 1 + 256);
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.p_full[i][0], 128);
+      mbar_init(&sm.p_full[i][1], 128);
+      mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.o_free[i], 128);
+      for (int j = 0; j < 2; ++j) {
+        mbar_init(&sm.s_full[i][j], 1);
+        mbar_init(&sm.s_empty[i][j], 128);
+      }
+    }
+    mbar_init(&sm.q_empty, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
+    }
+    for (int i = 0; i < kDecRingSlots; ++i) {
+      mbar_init(&sm.dec_full[i], 2);
+      mbar_init(&sm.dec_empty[i], 1);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wctx{&sm.abort_flag, p.status};
+  const bool gated = p.mode == kModeGated;
+
+  if (warp == 0) {
+    // ============================ Q/K producer ============================
+    if (lane == 0) {
+      tma_prefetch_desc(&mapQ);
+      tma_prefetch_desc(&mapK);
+      tma_prefetch_desc(&mapV);
+    }
+    int ks = 0;
+    uint32_t kph = 0;
+    bool ok = true;
+    int n = 0;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
+      const int ub = n & 1;
+      PfSched& sc = sm.sched[ub];
+      if (lane == 0) ok = mbar_wait(&sm.sched_empty[ub], ((n >> 1) & 1) ^ 1u, wctx);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      pf_build_sched(p, u, sc, lane);
+      if (lane == 0) {
+        mbar_arrive(&sm.sched_full[ub]);
+        ok = mbar_wait(&sm.q_empty, (n & 1) ^ 1u, wctx);
+        if (ok) {
+          for (int t = 0; t < 2; ++t) {
+            const int nv = sc.seg_valid[2 * t] + sc.seg_valid[2 * t + 1];
+            mbar_arrive_expect_tx(&sm.q_full[t], nv * 2 * 8192);
+            for (int h = 0; h < 2; ++h) {
+              const int s = 2 * t + h;
+              if (!sc.seg_valid[s]) continue;
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d(sm.q[t] + c * 16384 + h * 8192, &mapQ, &sm.q_full[t], c * 64,
+                            sc.seg_head[s], sc.seg_row0[s], sc.b);
+            }
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
+        bool good = true;
+        if (lane == 0) good = mbar_wait(&sm.k_empty[ks], kph ^ 1u, wctx);
+        good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+        if (!good) return false;
+        if (!is_col) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.k_full[ks], kTileBytes);
+            tma_load_4d(sm.k[ks], &mapK, &sm.k_full[ks], 0, sc.g, kt * 64, sc.b);
+            tma_load_4d(sm.k[ks] + 8192, &mapK, &sm.k_full[ks], 64, sc.g, kt * 64, sc.b);
+          }
+        } else {
+          pf_gather_rows(sc, kt, p.k, p.ksb, p.kss, p.ksh, sm.k[ks], lane);
+          if (lane == 0) mbar_arrive(&sm.k_full[ks]);
+        }
+        if (++ks == kKStages) { ks = 0; kph ^= 1u; }
+        return true;
+      };
+      ok = pf_for_each(sc, body);
+    }
+    if (!ok && lane == 0)
+      for (int i = 0; i < kKStages; ++i) mbar_wait_short(&sm.k_full[i], 0);
+  } else if (warp == 2) {
+    // ============================= V producer =============================
+    int vs = 0;
+    uint32_t vph = 0;
+    int dslot = 0;
+    uint32_t dph = 0;
+    bool ok = true;
+    int n = 0;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
+      const int ub = n & 1;
+      PfSched& sc = sm.sched[ub];
+      if (lane == 0) ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
+        bool good = true;
+        int need = 1;
+        if (gated) {
+          if (lane == 0) {
+            good = mbar_wait(&sm.dec_full[dslot], dph, wctx);
+            if (good) {
+              need = sm.dec_val[dslot][0] | sm.dec_val[dslot][1];
+              mbar_arrive(&sm.dec_empty[dslot]);
+            }
+          }
+          if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
+          good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+          need = __shfl_sync(0xffffffffu, need, 0);
+          if (!good) return false;
+          if (!need) return true;
+        }
+        if (lane == 0) good = mbar_wait(&sm.v_empty[vs], vph ^ 1u, wctx);
+        good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+        if (!good) return false;
+        if (!is_col) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.v_full[vs], kTileBytes);
+            tma_load_4d(sm.v[vs], &mapV, &sm.v_full[vs], 0, sc.g, kt * 64, sc.b);
+            tma_load_4d(sm.v[vs] + 8192, &mapV, &sm.v_full[vs], 64, sc.g, kt * 64, sc.b);
+          }
+        } else {
+          pf_gather_rows(sc, kt, p.v, p.vsb, p.vss, p.vsh, sm.v[vs], lane);
+          if (lane == 0) mbar_arrive(&sm.v_full[vs]);
+        }
+        if (++vs == kVStages) { vs = 0; vph ^= 1u; }
+        return true;
+      };
+      ok = pf_for_each(sc, body);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.sched_empty[ub]);
+    }
+    if (!ok && lane == 0)
+      for (int i = 0; i < kVStages; ++i) mbar_wait_short(&sm.v_full[i], 0);
+  } else if (warp == 1) {
+    // ============================= MMA issuer =============================
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16(128, 64, 0);
+      const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0;
+      int sbuf[2] = {0, 0};
+      uint32_t sph[2][2] = {{0, 0}, {0, 0}};
+      uint32_t pph[2][2] = {{0, 0}, {0, 0}};
+      int pslot[2] = {0, 0};
+      uint32_t ofph[2] = {0, 0};
+      bool ok = true;
+      int n = 0;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
+        const int ub = n & 1;
+        PfSched& sc = sm.sched[ub];
+        ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
+        if (!ok) break;
+        ok = mbar_wait(&sm.q_full[0], n & 1, wctx) && mbar_wait(&sm.q_full[1], n & 1, wctx);
+        if (!ok) break;
+        int pv_started[2] = {0, 0};
+        int ofree_waited[2] = {0, 0};
+        int prev_act = 0;  // bit t: tile t took part in the previous item
+        auto do_pv = [&](int act) -> bool {
+          int flag[2] = {0, 0};
+          for (int t = 0; t < 2; ++t) {
+            if (!((act >> t) & 1)) continue;
+            const int sl = pslot[t];
+            if (!mbar_wait(&sm.p_full[t][sl], pph[t][sl], wctx)) return false;
+            pph[t][sl] ^= 1u;
+            flag[t] = sm.pv_flag[t][sl];
+            pslot[t] ^= 1;
+          }
+          if (!(flag[0] | flag[1])) return true;
+          if (!mbar_wait(&sm.v_full[vs], vph, wctx)) return false;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (!flag[t]) continue;
+            if (!ofree_waited[t]) {
+              if (!mbar_wait(&sm.o_free[t], ofph[t] ^ 1u, wctx)) return false;
+              ofph[t] ^= 1u;
+              ofree_waited[t] = 1;
+              tc_fence_after();
+            }
+            const uint32_t d_tmem = tmem + t * 256 + 128;
+            const uint32_t pa = smem_u32(sm.p[t]);
+            const uint32_t va = smem_u32(sm.v[vs]);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sdesc_sw128(pa + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(va + kk * 2048, 8192, 1024);
+              umma_ss(d_tmem, ad, bd, idesc_pv, (pv_started[t] | kk) ? 1u : 0u);
+            }
+            pv_started[t] = 1;
+            umma_commit(&sm.pv_done[t]);
+          }
+          umma_commit(&sm.v_empty[vs]);
+          if (++vs == kVStages) { vs = 0; vph ^= 1u; }
+          return true;
+        };
+        auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
+          const int act = ((mem & 3) ? 1 : 0) | ((mem & 12) ? 2 : 0);
+          if (!mbar_wait(&sm.k_full[ks], kph, wctx)) return false;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (!((act >> t) & 1)) continue;
+            const int bsel = sbuf[t];
+            if (!mbar_wait(&sm.s_empty[t][bsel], sph[t][bsel] ^ 1u, wctx)) return false;
+            sph[t][bsel] ^= 1u;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + t * 256 + bsel * 64;
+            const uint32_t qa = smem_u32(sm.q[t]);
+            const uint32_t ka = smem_u32(sm.k[ks]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+              umma_ss(d_tmem, ad, bd, idesc_qk, kk ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[t][bsel]);
+            sbuf[t] ^= 1;
+          }
+          umma_commit(&sm.k_empty[ks]);
+          if (++ks == kKStages) { ks = 0; kph ^= 1u; }
+          if (prev_act && !do_pv(prev_act)) return false;
+          prev_act = act;
+          return true;
+        };
+        ok = pf_for_each(sc, body);
+        if (ok && prev_act) ok = do_pv(prev_act);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!ofree_waited[t]) {
+            ok = mbar_wait(&sm.o_free[t], ofph[t] ^ 1u, wctx);
+            ofph[t] ^= 1u;
+          }
+        }
+        umma_commit(&sm.q_empty);
+        mbar_arrive(&sm.sched_empty[ub]);
+      }
+      // make sure every issued tcgen05 op has finished before TMEM is freed
+      umma_commit(&sm.q_empty);
+      mbar_wait_short(&sm.q_empty, (n & 1));
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================ softmax warpgroups ============================
+    const int t = (warp - 4) >> 2;        // tile
+    const int r = tid - 128 - 128 * t;    // row in tile == TMEM lane
+    const int quarter = (warp & 3);
+    const int hseg = r >> 6;              // 0/1: segment within tile
+    const int seg = 2 * t + hseg;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 256;
+    const int bar_id = 1 + t;
+    const float NEG = -INFINITY;
+    int sbuf = 0;
+    uint32_t sphase = 0;  // bit b: phase of S buffer b
+    int dslot = 0;
+    uint32_t dph = 0;
+    int dbuf = 0;
+    int pslot = 0;        // p_full / pv_flag ring slot of this tile
+    uint32_t pv_total = 0;  // PVs issued for this tile so far (pv_done phases)
+    bool ok = true;
+    int n = 0;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
+      const int ub = n & 1;
+      PfSched& sc = sm.sched[ub];
+      ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
+      if (!ok) break;
+      const int my_valid = sc.seg_valid[seg];
+      const int my_row = sc.seg_row0[seg] + (r & 63);
+      float m_used = NEG, l = 0.f;
+      int npv = 0;
+      auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
+        const bool tile_act = (mem >> (2 * t)) & 3;
+        if (!tile_act) {
+          if (gated) {
+            if (tid == 128 + 128 * t) {
+              if (!mbar_wait(&sm.dec_empty[dslot], dph ^ 1u, wctx)) return false;
+              sm.dec_val[dslot][t] = 0;
+              mbar_arrive(&sm.dec_full[dslot]);
+            }
+            if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
+          }
+          return true;
+        }
+        const bool seg_act = ((mem >> seg) & 1) && my_row < p.Sq;
+        if (!mbar_wait(&sm.s_full[t][sbuf], (sphase >> sbuf) & 1u, wctx)) return false;
+        sphase ^= 1u << sbuf;
+        tc_fence_after();
+        float s[64];
+        tmem_ld32(lane_addr + sbuf * 64, s);
+        tmem_ld32(lane_addr + sbuf * 64 + 32, s + 32);
+        tc_fence_before();
+        mbar_arrive(&sm.s_empty[t][sbuf]);
+        sbuf ^= 1;
+        // ---- masks
+        float rmax = NEG;
+        if (!is_col) {
+          const int key0 = kt * 64;
+          const bool need =
+              (p.causal && key0 + 63 > my_row + p.causal_off) || (key0 + 64 > p.Sk);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            bool vis = seg_act;
+            if (need) {
+              const int key = key0 + c;
+              vis = vis && key < p.Sk && (!p.causal || key <= my_row + p.causal_off);
+            }
+            s[c] = vis ? s[c] : NEG;
+            rmax = fmaxf(rmax, s[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int e = kt * 64 + c;
+            bool vis = seg_act && e < sc.n_cols && ((sc.colmask[e] >> seg) & 1);
+            if (vis && p.causal) vis = sc.col[e] <= my_row + p.causal_off;
+            s[c] = vis ? s[c] : NEG;
+            rmax = fmaxf(rmax, s[c]);
+          }
+        }
+        bool my_keep = seg_act;
+        bool tile_keep = true;
+        if (gated) {
+          // exact block max of each 64 x 64 sub-tile (BSFA Figure 2a)
+          float wm = rmax;
+          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 16));
+          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 8));
+          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 4));
+          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 2));
+          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 1));
+          if (lane == 0) sm.red[t][dbuf][quarter] = wm;
+          named_bar_sync(bar_id, 128);
+          bool keep2[2];
+          for (int hh = 0; hh < 2; ++hh) {
+            const int sgi = 2 * t + hh;
+            const float bmax = fmaxf(sm.red[t][dbuf][2 * hh], sm.red[t][dbuf][2 * hh + 1]);
+            const bool act = (mem >> sgi) & 1;
+            const float smax = bmax * p.scale;
+            const bool diag = kt == sc.seg_qb[sgi];
+            keep2[hh] = act && (diag || smax >= sc.seg_T[sgi]);
+            if (act && (r == 64 * hh)) {
+              const int64_t oi =
+                  ((static_cast<int64_t>(sc.b) * p.Hq + sc.seg_head[sgi]) * p.nqb +
+                   sc.seg_qb[sgi]) * p.nqb + kt;
+              if (p.smax_out) p.smax_out[oi] = smax;
+              if (p.keep_out) p.keep_out[oi] = keep2[hh] ? 1 : 0;
+            }
+          }
+          dbuf ^= 1;
+          my_keep = hseg ? keep2[1] : keep2[0];
+          tile_keep = keep2[0] || keep2[1];
+          if (r == 0) {
+            if (!mbar_wait(&sm.dec_empty[dslot], dph ^ 1u, wctx)) return false;
+            sm.dec_val[dslot][t] = tile_keep ? 1 : 0;
+            mbar_arrive(&sm.dec_full[dslot]);
+          }
+          if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
+        }
+        if (!tile_keep) {
+          if (r == 0) sm.pv_flag[t][pslot] = 0;
+          mbar_arrive(&sm.p_full[t][pslot]);
+          pslot ^= 1;
+          return true;
+        }
+        // ---- online softmax (log2 domain, lazy rescale)
+        float alpha = 1.f;
+        bool resc = false;
+        if (my_keep && rmax != NEG) {
+          const float mrow = rmax * p.scale_log2;
+          if (mrow > m_used + 8.f) {
+            alpha = ex2_approx(m_used - mrow);
+            resc = true;
+            m_used = mrow;
+          }
+        }
+        const float mu = (m_used == NEG) ? 0.f : m_used;
+        float psum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float p0 = 0.f, p1 = 0.f;
+          if (my_keep) {
+            p0 = ex2_approx(fmaf(s[c], p.scale_log2, -mu));
+            p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -mu));
+          }
+          psum += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + psum;
+        if (npv > 0) {
+          if (!mbar_wait(&sm.pv_done[t], (pv_total - 1) & 1, wctx)) return false;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, resc)) {
+            float ob[32];
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              tmem_ld32(lane_addr + 128 + c * 32, ob);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ob[i] *= alpha;
+              tmem_st32(lane_addr + 128 + c * 32, ob);
+            }
+          }
+        }
+        // P row -> shared memory (K-major, 128B swizzle)
+        const uint32_t prow = smem_u32(sm.p[t]);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, cc)),
+                       "r"(pk[cc * 4]), "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]),
+                       "r"(pk[cc * 4 + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (r == 0) sm.pv_flag[t][pslot] = 1;
+        mbar_arrive(&sm.p_full[t][pslot]);
+        pslot ^= 1;
+        ++npv;
+        ++pv_total;
+        return true;
+      };
+      ok = pf_for_each(sc, body);
+      if (!ok) break;
+      // ---- epilogue: o = O / l, lse = ln(sum)
+      const bool store = my_valid && my_row < p.Sq;
+      const int head = sc.seg_head[seg];
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      if (npv > 0) {
+        if (!mbar_wait(&sm.pv_done[t], (pv_total - 1) & 1, wctx)) { ok = false; break; }
+        tc_fence_after();
+        float ob[32];
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(lane_addr + 128 + c * 32, ob);
+          if (store) {
+            const int64_t off = sc.b * p.osb + static_cast<int64_t>(my_row) * p.oss + head * p.osh + c * 32;
+            if (p.o_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(ob[4 * i] * inv_l, ob[4 * i + 1] * inv_l,
+                                     ob[4 * i + 2] * inv_l, ob[4 * i + 3] * inv_l);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_bf16x2(ob[8 * i] * inv_l, ob[8 * i + 1] * inv_l),
+                                    pack_bf16x2(ob[8 * i + 2] * inv_l, ob[8 * i + 3] * inv_l),
+                                    pack_bf16x2(ob[8 * i + 4] * inv_l, ob[8 * i + 5] * inv_l),
+                                    pack_bf16x2(ob[8 * i + 6] * inv_l, ob[8 * i + 7] * inv_l));
+            }
+          }
+        }
+      } else if (store) {
+        const int64_t off = sc.b * p.osb + static_cast<int64_t>(my_row) * p.oss + head * p.osh;
+        for (int c = 0; c < 128; c += 4) {
+          if (p.o_f32)
+            *reinterpret_cast<float4*>(static_cast<float*>(p.o) + off + c) = make_float4(0, 0, 0, 0);
+          else
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.o) + off + c) = make_uint2(0, 0);
+        }
+      }
+      if (store)
+        p.lse[(static_cast<int64_t>(sc.b) * p.Hq + head) * p.Sq + my_row] =
+            l > 0.f ? (m_used + lg2_approx(l)) * 0.69314718055994531f : NEG;
+      tc_fence_before();
+      mbar_arrive(&sm.o_free[t]);
+      mbar_arrive(&sm.sched_empty[ub]);
+    }
+  }
+  // warp 3 idles (reserved)
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sbfa

@@ -1,0 +1,552 @@
+// Host side of libsbfa: argument validation, TMA descriptor encoding and
+// kernel launches behind the C ABI declared in include/sbfa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "sbfa.h"
+#include "kernel_convert.cuh"
+#include "kernel_decode.cuh"
+#include "kernel_prefill.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sbfa_status fail(sbfa_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+sbfa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SBFA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define SBFA_CUDA(call)                                 \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no libcuda link).
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D map over a (B, S, H, 128) bf16 view: dims {D, H, S, B}; box
+// {64, 1, box_rows, 1}; 128-byte swizzle; out-of-range rows read as zero.
+sbfa_status encode_bshd(CUtensorMap* map, const sbfa_t4& t, int B, int S, int H, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return fail(SBFA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const int64_t sh = H > 1 ? t.sh : 128;
+  const int64_t ss = S > 1 ? t.ss : sh * H;
+  const int64_t sb = B > 1 ? t.sb : ss * S;
+  cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(sh * 2), static_cast<cuuint64_t>(ss * 2),
+                           static_cast<cuuint64_t>(sb * 2)};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SBFA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SBFA_OK;
+}
+
+struct DevInfo {
+  int sms = 0;
+};
+
+sbfa_status dev_info(DevInfo* di) {
+  static DevInfo cache[64];
+  int dev = 0;
+  SBFA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(SBFA_ERR_UNSUPPORTED, "device index %d", dev);
+  if (cache[dev].sms == 0) {
+    cudaDeviceProp prop;
+    SBFA_CUDA(cudaGetDeviceProperties(&prop, dev));
+    if (prop.major != 10)
+      return fail(SBFA_ERR_UNSUPPORTED, "needs an sm_100 GPU (found sm_%d%d)", prop.major,
+                  prop.minor);
+    cache[dev].sms = prop.multiProcessorCount;
+  }
+  *di = cache[dev];
+  return SBFA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sbfa_status check_view(const sbfa_t4& t, const char* name, bool need_tma) {
+  if (!t.ptr) return fail(SBFA_ERR_INVALID_ARG, "%s: null pointer", name);
+  if (!aligned16(t.ptr)) return fail(SBFA_ERR_INVALID_ARG, "%s: base not 16-byte aligned", name);
+  if (t.sb < 0 || t.ss < 0 || t.sh < 0)
+    return fail(SBFA_ERR_INVALID_ARG, "%s: negative stride", name);
+  if (need_tma && ((t.sb % 8) || (t.ss % 8) || (t.sh % 8)))
+    return fail(SBFA_ERR_INVALID_ARG, "%s: strides must be multiples of 8 elements", name);
+  return SBFA_OK;
+}
+
+sbfa_status check_shape(const sbfa_shape* s) {
+  if (!s) return fail(SBFA_ERR_INVALID_ARG, "shape is null");
+  if (s->B <= 0 || s->Sq <= 0 || s->Sk <= 0 || s->Hq <= 0 || s->Hkv <= 0)
+    return fail(SBFA_ERR_INVALID_ARG, "non-positive size (B=%d Sq=%d Sk=%d Hq=%d Hkv=%d)", s->B,
+                s->Sq, s->Sk, s->Hq, s->Hkv);
+  if (s->D != 128) return fail(SBFA_ERR_UNSUPPORTED, "head dim %d (only 128)", s->D);
+  if (s->Hq % s->Hkv) return fail(SBFA_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (s->causal != 0 && s->causal != 1) return fail(SBFA_ERR_INVALID_ARG, "causal must be 0/1");
+  if (s->Sk > sbfa::kMaxKT * 64) return fail(SBFA_ERR_UNSUPPORTED, "Sk > %d", sbfa::kMaxKT * 64);
+  return SBFA_OK;
+}
+
+float eff_scale(const sbfa_shape* s) {
+  return s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(s->D));
+}
+
+#define SBFA_TRY(x)                \
+  do {                             \
+    sbfa_status st_ = (x);         \
+    if (st_ != SBFA_OK) return st_; \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// prefill launcher (tcgen05 kernel)
+// ---------------------------------------------------------------------------
+sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sbfa_t4& q,
+                           const sbfa_t4& k, const sbfa_t4& v, cudaStream_t stream) {
+  DevInfo di;
+  SBFA_TRY(dev_info(&di));
+  p.B = s->B;
+  p.Sq = s->Sq;
+  p.Sk = s->Sk;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.G = s->Hq / s->Hkv;
+  p.hp = (p.G % 4 == 0) ? 4 : (p.G % 2 == 0 ? 2 : 1);
+  p.subs_per_unit = 4 / p.hp;
+  p.n_sub = (s->Sq + 63) / 64;
+  p.n_hgrp = p.G / p.hp;
+  p.n_subgrp = (p.n_sub + p.subs_per_unit - 1) / p.subs_per_unit;
+  const int64_t units = static_cast<int64_t>(p.B) * p.Hkv * p.n_hgrp * p.n_subgrp;
+  if (units > 0x7fffffff) return fail(SBFA_ERR_UNSUPPORTED, "too many work units");
+  p.n_units = static_cast<int>(units);
+  p.n_kt = (s->Sk + 63) / 64;
+  p.causal = s->causal;
+  p.causal_off = s->Sk - s->Sq;
+  p.scale = eff_scale(s);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.k = static_cast<const __nv_bfloat16*>(k.ptr);
+  p.v = static_cast<const __nv_bfloat16*>(v.ptr);
+  p.ksb = k.sb; p.kss = k.ss; p.ksh = k.sh;
+  p.vsb = v.sb; p.vss = v.ss; p.vsh = v.sh;
+  CUtensorMap mq, mk, mv;
+  SBFA_TRY(encode_bshd(&mq, q, s->B, s->Sq, s->Hq, 64));
+  SBFA_TRY(encode_bshd(&mk, k, s->B, s->Sk, s->Hkv, 64));
+  SBFA_TRY(encode_bshd(&mv, v, s->B, s->Sk, s->Hkv, 64));
+  const size_t smem = sizeof(sbfa::PfSmem) + 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  SBFA_CUDA(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::prefill_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr_set[dev] = true;
+  }
+  const int grid = std::min(p.n_units, di.sms);
+  sbfa::prefill_kernel<<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
+}
+
+sbfa_status check_outputs(const sbfa_t4& o, const float* lse) {
+  SBFA_TRY(check_view(o, "o", false));
+  if (!lse) return fail(SBFA_ERR_INVALID_ARG, "lse: null pointer");
+  return SBFA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// decode launcher (split-KV kernel)
+// ---------------------------------------------------------------------------
+struct DecodeWs {
+  int* ticket;
+  float* part;
+  float* lse;
+};
+
+size_t decode_ws_bytes(int npairs, int grid) {
+  const size_t tick = ((static_cast<size_t>(npairs) * 4 + 255) / 256) * 256;
+  const size_t part = static_cast<size_t>(grid) * 2 * sbfa::kDecRows * sbfa::kDecD * 4;
+  const size_t lse = static_cast<size_t>(grid) * 2 * sbfa::kDecRows * 4;
+  return tick + part + lse;
+}
+
+sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa_t4& q,
+                          const sbfa_t4* kA, const sbfa_t4* vA, int S_A, int causal_A,
+                          const sbfa_t4* kB, const sbfa_t4* vB, const sbfa_table* tb, void* ws,
+                          size_t ws_bytes, const sbfa_t4& o, float* lse, int32_t* status,
+                          cudaStream_t stream) {
+  DevInfo di;
+  SBFA_TRY(dev_info(&di));
+  const int G = s->Hq / s->Hkv;
+  const int npairs = s->B * s->Hkv;
+  if (npairs > sbfa::kDecMaxPairs)
+    return fail(SBFA_ERR_UNSUPPORTED, "B*Hkv = %d > %d", npairs, sbfa::kDecMaxPairs);
+  p.B = s->B; p.Sq = s->Sq; p.Hq = s->Hq; p.Hkv = s->Hkv; p.G = G; p.rows = s->Sq * G;
+  p.scale_log2 = eff_scale(s) * 1.4426950408889634f;
+  p.q = static_cast<const __nv_bfloat16*>(q.ptr); p.qsb = q.sb; p.qss = q.ss; p.qsh = q.sh;
+  p.o = static_cast<__nv_bfloat16*>(o.ptr); p.osb = o.sb; p.oss = o.ss; p.osh = o.sh;
+  p.lse = lse;
+  p.status = status;
+  CUtensorMap mKA, mVA, mKB, mVB;
+  p.has_A = kA != nullptr;
+  p.S_A = S_A;
+  p.causal_A = causal_A;
+  p.has_B = tb != nullptr;
+  if (kA) {
+    SBFA_TRY(encode_bshd(&mKA, *kA, s->B, S_A, s->Hkv, 64));
+    SBFA_TRY(encode_bshd(&mVA, *vA, s->B, S_A, s->Hkv, 64));
+  }
+  if (tb) {
+    SBFA_TRY(encode_bshd(&mKB, *kB, s->B, s->Sk, s->Hkv, 64));
+    SBFA_TRY(encode_bshd(&mVB, *vB, s->B, s->Sk, s->Hkv, 64));
+    p.S_B = s->Sk;
+    p.kv_block = tb->kv_block;
+    p.nmax = tb->nmax;
+    p.n_kb = (s->Sk + tb->kv_block - 1) / tb->kv_block;
+    p.idx = tb->idx;
+    p.tsb = tb->sb;
+    p.tsh = tb->sh;
+  } else {
+    p.S_B = 0; p.kv_block = 64; p.nmax = 0; p.n_kb = 0; p.idx = nullptr; p.tsb = p.tsh = 0;
+  }
+  if (!kA) { mKA = mKB; mVA = mVB; }
+  if (!tb) { mKB = mKA; mVB = mVA; }
+  const int grid = di.sms;
+  if (ws) {
+    const size_t need = decode_ws_bytes(npairs, grid);
+    if (ws_bytes < need)
+      return fail(SBFA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    if (!aligned16(ws)) return fail(SBFA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    const size_t tick = ((static_cast<size_t>(npairs) * 4 + 255) / 256) * 256;
+    p.ws_ticket = reinterpret_cast<int*>(w);
+    p.ws_part = reinterpret_cast<float*>(w + tick);
+    p.ws_lse = reinterpret_cast<float*>(w + tick +
+                                        static_cast<size_t>(grid) * 2 * sbfa::kDecRows *
+                                            sbfa::kDecD * 4);
+    p.pair_mode = 0;
+  } else {
+    p.ws_ticket = nullptr; p.ws_part = nullptr; p.ws_lse = nullptr;
+    p.pair_mode = 1;
+  }
+  const size_t smem = sizeof(sbfa::DecSmem) + 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  SBFA_CUDA(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::decode_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr_set[dev] = true;
+  }
+  sbfa::decode_kernel<<<grid, sbfa::kDecThreads, smem, stream>>>(mKA, mVA, mKB, mVB, p);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
+}
+
+bool decode_shape(const sbfa_shape* s) {
+  return s->Sq * (s->Hq / s->Hkv) <= sbfa::kDecRows;
+}
+
+sbfa_status check_table(const sbfa_table* t, const sbfa_shape* s, bool prefill) {
+  if (!t || !t->idx) return fail(SBFA_ERR_INVALID_ARG, "table: null");
+  if (t->nmax < 0) return fail(SBFA_ERR_INVALID_ARG, "table: nmax < 0");
+  if (t->sb < 0 || t->sh < 0 || t->sqb < 0) return fail(SBFA_ERR_INVALID_ARG, "table: negative stride");
+  if (t->q_block <= 0) return fail(SBFA_ERR_INVALID_ARG, "table: q_block <= 0");
+  const int kb = t->kv_block;
+  if (prefill) {
+    if (kb != 64 && kb != 128 && kb != 256)
+      return fail(SBFA_ERR_UNSUPPORTED, "kv_block %d (prefill kernel takes 64/128/256)", kb);
+    if (t->q_block % 64 && t->q_block < s->Sq)
+      return fail(SBFA_ERR_UNSUPPORTED, "q_block %d: must be a multiple of 64 or >= Sq",
+                  t->q_block);
+  } else {
+    if (kb != 16 && kb != 32 && kb != 64 && kb != 128 && kb != 256)
+      return fail(SBFA_ERR_UNSUPPORTED, "kv_block %d", kb);
+    if (t->nmax > sbfa::kDecMaxEntries)
+      return fail(SBFA_ERR_UNSUPPORTED, "nmax %d > %d", t->nmax, sbfa::kDecMaxEntries);
+  }
+  return SBFA_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* sbfa_last_error(void) { return g_last_error.c_str(); }
+
+const char* sbfa_version(void) { return "sbfa 0.1 (sm_100a)"; }
+
+sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                     const sbfa_table* table, sbfa_t4 o, float* lse, int32_t* status,
+                     sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  const bool dec = decode_shape(shape) && table && table->q_block >= shape->Sq;
+  SBFA_TRY(check_table(table, shape, !dec));
+  if (dec) {
+    sbfa::DecodeParams p{};
+    return launch_decode(p, shape, q, nullptr, nullptr, 0, 0, &k, &v, table, nullptr, 0, o,
+                         lse, status, reinterpret_cast<cudaStream_t>(stream));
+  }
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeTable;
+  p.o = o.ptr; p.osb = o.sb; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.idx = table->idx; p.tsb = table->sb; p.tsh = table->sh; p.tsqb = table->sqb;
+  p.nmax = table->nmax; p.q_block = table->q_block; p.kv_block = table->kv_block;
+  p.n_kb = (shape->Sk + table->kv_block - 1) / table->kv_block;
+  p.status = status;
+  return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_fwd_dense(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v, sbfa_t4 o,
+                           float* lse, int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  if (decode_shape(shape)) {
+    sbfa::DecodeParams p{};
+    return launch_decode(p, shape, q, &k, &v, shape->Sk, shape->causal, nullptr, nullptr,
+                         nullptr, nullptr, 0, o, lse, status,
+                         reinterpret_cast<cudaStream_t>(stream));
+  }
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeDense;
+  p.o = o.ptr; p.osb = o.sb; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.status = status;
+  return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_fwd_partials(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                              const sbfa_table* table, float* o_parts, float* lse_parts,
+                              int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_table(table, shape, true));
+  if (!o_parts || !lse_parts) return fail(SBFA_ERR_INVALID_ARG, "partials: null output");
+  if (!aligned16(o_parts)) return fail(SBFA_ERR_INVALID_ARG, "o_parts not 16-byte aligned");
+  const int64_t per_o = static_cast<int64_t>(shape->B) * shape->Sq * shape->Hq * shape->D;
+  const int64_t per_l = static_cast<int64_t>(shape->B) * shape->Hq * shape->Sq;
+  for (int n = 0; n < table->nmax; ++n) {
+    sbfa::PrefillParams p{};
+    p.mode = sbfa::kModeTable;
+    p.o = o_parts + n * per_o;
+    p.osb = static_cast<int64_t>(shape->Sq) * shape->Hq * shape->D;
+    p.oss = static_cast<int64_t>(shape->Hq) * shape->D;
+    p.osh = shape->D;
+    p.o_f32 = 1;
+    p.lse = lse_parts + n * per_l;
+    p.idx = table->idx + n; p.tsb = table->sb; p.tsh = table->sh; p.tsqb = table->sqb;
+    p.nmax = 1; p.q_block = table->q_block; p.kv_block = table->kv_block;
+    p.n_kb = (shape->Sk + table->kv_block - 1) / table->kv_block;
+    p.status = status;
+    SBFA_TRY(launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream)));
+  }
+  return SBFA_OK;
+}
+
+sbfa_status sbfa_combine(int32_t n_parts, int32_t B, int32_t Sq, int32_t Hq, int32_t D,
+                         const float* o_parts, const float* lse_parts, sbfa_t4 o, float* lse,
+                         sbfa_stream_t stream) {
+  g_last_error.clear();
+  if (n_parts < 0 || B <= 0 || Sq <= 0 || Hq <= 0) return fail(SBFA_ERR_INVALID_ARG, "bad sizes");
+  if (D != 128) return fail(SBFA_ERR_UNSUPPORTED, "head dim %d (only 128)", D);
+  if ((n_parts > 0 && (!o_parts || !lse_parts)) || !lse || !o.ptr)
+    return fail(SBFA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(o_parts)) return fail(SBFA_ERR_INVALID_ARG, "o_parts not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(o.ptr) & 7u) || (o.sb % 4) || (o.ss % 4) || (o.sh % 4))
+    return fail(SBFA_ERR_INVALID_ARG, "o: needs 8-byte aligned rows");
+  const int64_t rows = static_cast<int64_t>(B) * Sq * Hq;
+  const int threads = 256;
+  const int64_t blocks = (rows * 32 + threads - 1) / threads;
+  sbfa::combine_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                         reinterpret_cast<cudaStream_t>(stream)>>>(
+      n_parts, B, Sq, Hq, o_parts, lse_parts, static_cast<__nv_bfloat16*>(o.ptr), o.sb, o.ss,
+      o.sh, lse);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
+}
+
+size_t sbfa_decode_workspace_size(int32_t B, int32_t Hkv, int32_t Sq, int32_t Hq) {
+  (void)Sq;
+  (void)Hq;
+  DevInfo di;
+  if (dev_info(&di) != SBFA_OK) return 0;
+  return decode_ws_bytes(B * Hkv, di.sms);
+}
+
+sbfa_status sbfa_speculative_sparse(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k_spec,
+                                    sbfa_t4 v_spec, int32_t S_spec, int32_t causal_spec,
+                                    sbfa_t4 k, sbfa_t4 v, const sbfa_table* missed, void* ws,
+                                    size_t ws_bytes, sbfa_t4 o, float* lse, int32_t* status,
+                                    sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", false));
+  SBFA_TRY(check_view(k_spec, "k_spec", true));
+  SBFA_TRY(check_view(v_spec, "v_spec", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  if (S_spec <= 0) return fail(SBFA_ERR_INVALID_ARG, "S_spec <= 0");
+  if (causal_spec != 0 && causal_spec != 1) return fail(SBFA_ERR_INVALID_ARG, "causal_spec");
+  if (!decode_shape(shape))
+    return fail(SBFA_ERR_UNSUPPORTED, "Sq * Hq/Hkv = %d > %d", shape->Sq * (shape->Hq / shape->Hkv),
+                sbfa::kDecRows);
+  SBFA_TRY(check_table(missed, shape, false));
+  if (missed->q_block < shape->Sq) return fail(SBFA_ERR_UNSUPPORTED, "missed->q_block < Sq");
+  if (!ws) return fail(SBFA_ERR_INVALID_ARG, "workspace is null");
+  sbfa::DecodeParams p{};
+  return launch_decode(p, shape, q, &k_spec, &v_spec, S_spec, causal_spec, &k, &v, missed, ws,
+                       ws_bytes, o, lse, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_fwd_gated(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                           const float* T, int32_t block, sbfa_t4 o, float* lse, float* smax_out,
+                           uint8_t* keep_out, int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  if (!T) return fail(SBFA_ERR_INVALID_ARG, "T is null");
+  if (block != 64) return fail(SBFA_ERR_UNSUPPORTED, "gate block %d (only 64)", block);
+  if (shape->Sq != shape->Sk || !shape->causal)
+    return fail(SBFA_ERR_UNSUPPORTED, "gated mode needs Sq == Sk and causal");
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeGated;
+  p.o = o.ptr; p.osb = o.sb; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.T = T;
+  p.nqb = (shape->Sq + 63) / 64;
+  p.smax_out = smax_out;
+  p.keep_out = keep_out;
+  p.status = status;
+  return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_convert_vertical_slash(const int32_t* q_seqlens, const int32_t* kv_seqlens,
+                                        const int32_t* vertical, int32_t nnz_v,
+                                        const int32_t* slash, int32_t nnz_s, int32_t B,
+                                        int32_t H, int32_t context_size, int32_t block_M,
+                                        int32_t block_N, int32_t causal, int32_t* block_count,
+                                        int32_t* block_offset, int32_t* column_count,
+                                        int32_t* column_index, int32_t* status,
+                                        sbfa_stream_t stream) {
+  g_last_error.clear();
+  if (!q_seqlens || !kv_seqlens || !vertical || !slash || !block_count || !block_offset ||
+      !column_count || !column_index)
+    return fail(SBFA_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || H <= 0 || context_size <= 0 || nnz_v < 0 || nnz_s < 0)
+    return fail(SBFA_ERR_INVALID_ARG, "bad sizes");
+  if (block_M != 64 || block_N != 64)
+    return fail(SBFA_ERR_UNSUPPORTED, "block_M = block_N = 64 only");
+  if (context_size > sbfa::kCvMaxWords * 32 * 64)
+    return fail(SBFA_ERR_UNSUPPORTED, "context_size too large");
+  const int nqb = (context_size + block_M - 1) / block_M;
+  const int64_t grid = static_cast<int64_t>(B) * H * nqb;
+  sbfa::convert_vs_kernel<<<static_cast<unsigned>(grid), sbfa::kCvThreads, 0,
+                            reinterpret_cast<cudaStream_t>(stream)>>>(
+      q_seqlens, kv_seqlens, vertical, nnz_v, slash, nnz_s, H, nqb, block_M, block_N, causal,
+      block_count, block_offset, column_count, column_index, status);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
+}
+
+sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                                    const int32_t* block_count, const int32_t* block_offset,
+                                    int32_t nnz_s, const int32_t* column_count,
+                                    const int32_t* column_index, int32_t nnz_v, int32_t block_M,
+                                    int32_t block_N, sbfa_t4 o, float* lse, int32_t* status,
+                                    sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  if (block_M != 64 || block_N != 64)
+    return fail(SBFA_ERR_UNSUPPORTED, "block_M = block_N = 64 only");
+  if (!block_count || !block_offset || !column_count || !column_index)
+    return fail(SBFA_ERR_INVALID_ARG, "null index array");
+  if (nnz_s < 0 || nnz_v < 0) return fail(SBFA_ERR_INVALID_ARG, "negative nnz");
+  if ((k.ss % 8) || (v.ss % 8)) return fail(SBFA_ERR_INVALID_ARG, "k/v row stride");
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeVS;
+  p.o = o.ptr; p.osb = o.sb; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.vs_bc = block_count; p.vs_bo = block_offset; p.nnz_s = nnz_s;
+  p.vs_cc = column_count; p.vs_ci = column_index; p.nnz_v = nnz_v;
+  p.vs_nqb = (shape->Sq + 63) / 64;
+  p.status = status;
+  return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_check_status(const int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  if (!status) return SBFA_OK;
+  int32_t h = 0;
+  SBFA_CUDA(cudaMemcpy(&h, status, sizeof(h), cudaMemcpyDeviceToHost));
+  if (h & SBFA_DEV_TIMEOUT) return fail(SBFA_ERR_TIMEOUT, "device status 0x%x", h);
+  if (h) return fail(SBFA_ERR_DEVICE, "device status 0x%x", h);
+  return SBFA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,229 @@
+/*
+ * sbfa.h -- C ABI of the block-sparse FlashAttention forward for NVIDIA B200
+ * (sm_100a).
+ *
+ * Every entry point is asynchronous on the given CUDA stream, returns an
+ * sbfa_status, allocates nothing and keeps no device state between calls.
+ * The caller owns every input, output and workspace buffer (device memory
+ * unless stated otherwise).  Argument errors are detected on the host and
+ * returned before any launch; sbfa_last_error() then gives a message.
+ * Problems only the device can see (a table entry outside the key range, a
+ * wait that timed out) never trap: the kernel skips the offending work and
+ * ORs an SBFA_DEV_* bit into the optional int32 device status word, which
+ * the caller zeroes and reads back (see sbfa_check_status).
+ *
+ * Common conventions
+ *   - Tensors use the (batch, seq, head, dim) layout of the
+ *     Incremental_FlashAttention README (Usage 1): q (B, Sq, Hq, D),
+ *     k and v (B, Sk, Hkv, D), o like q.  An sbfa_t4 gives the base pointer
+ *     and element strides of the first three dims; the last dim must be
+ *     contiguous.  Strides must be multiples of 8 elements and base pointers
+ *     16-byte aligned (TMA rules).  q, k, v and o are bf16.
+ *   - lse is fp32 (B, Hq, Sq), contiguous, natural log of the softmax
+ *     denominator.  A row that sees no key gets o = 0, lse = -inf (README,
+ *     Usage 1: an empty table is a neutral partial).
+ *   - D must be 128.  Hq must be a multiple of Hkv; query head h reads kv
+ *     head h / (Hq / Hkv).
+ *   - scale <= 0 selects 1/sqrt(D).
+ *   - causal masks keys with index > row + (Sk - Sq) (bottom-right
+ *     alignment).
+ */
+#ifndef SBFA_H_
+#define SBFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sbfa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  SBFA_OK = 0,
+  SBFA_ERR_INVALID_ARG = 1, /* bad pointer, shape, stride or alignment */
+  SBFA_ERR_UNSUPPORTED = 2, /* valid request this build does not serve (D != 128, ...) */
+  SBFA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  SBFA_ERR_DEVICE = 4,      /* the device status word reported a problem */
+  SBFA_ERR_TIMEOUT = 5      /* a kernel wait hit its time limit */
+} sbfa_status;
+
+/* Bits of the device status word. */
+#define SBFA_DEV_BAD_INDEX 0x1 /* table / index entry outside the key range: entry skipped */
+#define SBFA_DEV_TIMEOUT 0x2   /* a bounded barrier wait gave up: the CTA stopped early */
+#define SBFA_DEV_OVERFLOW 0x4  /* a per-row list exceeded the kernel's capacity: truncated */
+
+/* A (B, S, H, D) view: base pointer and element strides of B, S and H. */
+typedef struct {
+  void* ptr;
+  int64_t sb, ss, sh;
+} sbfa_t4;
+
+typedef struct {
+  int32_t B, Sq, Sk, Hq, Hkv, D;
+  float scale;    /* <= 0: 1/sqrt(D) */
+  int32_t causal; /* 0 or 1 */
+} sbfa_shape;
+
+/*
+ * Sparse block table (Incremental_FlashAttention README, Usage 1,
+ * generalised per (batch, kv-head, q-block)).  Row r of query head h in
+ * batch b uses idx[b*sb + (h/G)*sh + (r/q_block)*sqb + n], n < nmax.  Each
+ * entry j >= 0 names the keys [j*kv_block, (j+1)*kv_block) clipped to Sk;
+ * entries < 0 are padding; repeated entries count once; order does not
+ * matter.  sb = sh = sqb = 0 broadcasts one 1-D table (the README's form).
+ */
+typedef struct {
+  const int32_t* idx;
+  int64_t sb, sh, sqb;
+  int32_t nmax, q_block, kv_block;
+} sbfa_table;
+
+/*
+ * sbfa_fwd -- block-table attention forward.
+ * Source: Incremental_FlashAttention README, "What's in this fork" (sparse
+ * block-table forward) and Usage 1.  Each query row attends only to the keys
+ * of the blocks its table row lists (with the causal mask if shape->causal).
+ * Constraints: kv_block in {64, 128, 256}; q_block a multiple of 64 (or
+ * >= Sq); Sk <= 524288.  Decode shapes (Sq * Hq/Hkv <= 16 and one q-block)
+ * run on the split-KV decode kernel, which also takes kv_block 16 and 32.
+ * Outputs: o (bf16, like q), lse (fp32 [B, Hq, Sq]).
+ * status: optional device int32, SBFA_DEV_* bits are ORed in.
+ */
+sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                     const sbfa_table* table, sbfa_t4 o, float* lse, int32_t* status,
+                     sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_dense -- dense attention over all Sk keys (causal if asked).
+ * Source: the README's pass over the speculative K/V subset (Usage 2).
+ * Same layouts and limits as sbfa_fwd.
+ */
+sbfa_status sbfa_fwd_dense(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                           sbfa_t4 o, float* lse, int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_partials -- one (o, lse) per table entry.
+ * Source: README, Usage 3 (per-block partials for a caller-side combine).
+ * o_parts: fp32 [nmax, B, Sq, Hq, D] contiguous; lse_parts: fp32
+ * [nmax, B, Hq, Sq] contiguous.  Partial n attends the keys of entry n of
+ * each row's table (a padding entry gives o = 0, lse = -inf).
+ */
+sbfa_status sbfa_fwd_partials(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                              const sbfa_table* table, float* o_parts, float* lse_parts,
+                              int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_combine -- exact merge of partial results over disjoint key sets.
+ * Source: README, "What's in this fork" (FA(A u B) == Combine(FA(A),
+ * FA(B))) and Usage 2.  With M = max_p lse_p and w_p = exp(lse_p - M):
+ * lse = M + ln sum_p w_p, o = sum_p w_p o_p / sum_p w_p; all partials empty
+ * gives (0, -inf).
+ * o_parts: fp32 [n_parts, B, Sq, Hq, D] contiguous, lse_parts: fp32
+ * [n_parts, B, Hq, Sq] contiguous.  o: bf16 view (D contiguous), lse: fp32
+ * [B, Hq, Sq].  D must be 128.
+ */
+sbfa_status sbfa_combine(int32_t n_parts, int32_t B, int32_t Sq, int32_t Hq, int32_t D,
+                         const float* o_parts, const float* lse_parts, sbfa_t4 o, float* lse,
+                         sbfa_stream_t stream);
+
+/*
+ * sbfa_speculative_sparse -- fused two-pass speculative + sparse decode.
+ * Source: README, Usage 2.  One launch computes, per query row, attention
+ * over (a) all S_spec keys of (k_spec, v_spec), causal if causal_spec, and
+ * (b) the blocks of (k, v) listed in `missed` (no mask), merged by the LSE
+ * combine inside the kernel.  The result equals attention over the union.
+ * shape->Sk is the length of k/v; shape->causal is ignored.
+ * Limits: Sq * (Hq/Hkv) <= 16; missed->q_block >= Sq; missed->kv_block in
+ * {16, 32, 64, 128, 256}; B*Hkv <= 4096; missed->nmax <= 1024.
+ * ws/ws_bytes: device workspace of at least sbfa_decode_workspace_size()
+ * bytes, zero-filled before its first use (the kernel leaves its counters at
+ * zero when it completes).  Calls sharing one workspace must not overlap.
+ */
+sbfa_status sbfa_speculative_sparse(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k_spec,
+                                    sbfa_t4 v_spec, int32_t S_spec, int32_t causal_spec,
+                                    sbfa_t4 k, sbfa_t4 v, const sbfa_table* missed,
+                                    void* ws, size_t ws_bytes, sbfa_t4 o, float* lse,
+                                    int32_t* status, sbfa_stream_t stream);
+
+/* Workspace bytes the split-KV decode kernel needs on the current device. */
+size_t sbfa_decode_workspace_size(int32_t B, int32_t Hkv, int32_t Sq, int32_t Hq);
+
+/*
+ * sbfa_fwd_gated -- BSFA gated causal prefill.
+ * Source: Block Sparse Flash Attention, Abstract and Figure 2.  For head h
+ * and q-block i (64 rows) the kernel computes S = scale*Q_i K_j^T for every
+ * causal key block j <= i (64 keys), its exact block max s_max(h,i,j), and
+ * keeps the block iff j == i (the diagonal always runs) or
+ * s_max >= T[h*nQB + i].  Skipped blocks load no V_j and run no P V_j.
+ * Requires Sq == Sk, causal, block == 64.  T: fp32 [Hq, nQB], nQB =
+ * ceil(Sq/64); -inf keeps every block.
+ * smax_out (nullable): fp32 [B, Hq, nQB, nQB], written for j <= i.
+ * keep_out (nullable): uint8 [B, Hq, nQB, nQB], 1/0, written for j <= i.
+ */
+sbfa_status sbfa_fwd_gated(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                           const float* T, int32_t block, sbfa_t4 o, float* lse,
+                           float* smax_out, uint8_t* keep_out, int32_t* status,
+                           sbfa_stream_t stream);
+
+/*
+ * sbfa_convert_vertical_slash -- raw vertical/slash indices to block lists.
+ * Source: Sglang Sparse Flash Attention, Description and I/O contract
+ * (convert_vertical_slash_indexes).  For batch b, head h and q-block i with
+ * rows [m0, m1), m1 = min(m0 + block_M, q_len), d = kv_len - q_len:
+ *   - slash offset s covers keys [m0+d-s, m1-1+d-s] clipped to [0, kv_len);
+ *     block_offset[b,h,i,:] lists, ascending, the offsets j*block_N of every
+ *     key block meeting the union of these ranges; block_count their number;
+ *   - column_index[b,h,i,:] lists, ascending, the vertical columns
+ *     c < kv_len (and c <= m1-1+d if causal) that lie in no listed block;
+ *     column_count their number.
+ * Entries past a count are left unwritten.
+ * q_seqlens, kv_seqlens: int32 [B] (device).  vertical: int32 [B, H, nnz_v],
+ * slash: int32 [B, H, nnz_s], each row ascending and distinct, slash >= 0.
+ * Outputs (int32): block_count, column_count [B, H, nQB]; block_offset
+ * [B, H, nQB, nnz_s]; column_index [B, H, nQB, nnz_v]; nQB =
+ * ceil(context_size / block_M).  Requires block_M == block_N == 64.
+ */
+sbfa_status sbfa_convert_vertical_slash(const int32_t* q_seqlens, const int32_t* kv_seqlens,
+                                        const int32_t* vertical, int32_t nnz_v,
+                                        const int32_t* slash, int32_t nnz_s, int32_t B,
+                                        int32_t H, int32_t context_size, int32_t block_M,
+                                        int32_t block_N, int32_t causal, int32_t* block_count,
+                                        int32_t* block_offset, int32_t* column_count,
+                                        int32_t* column_index, int32_t* status,
+                                        sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_vertical_slash -- sparse attention over converted block lists.
+ * Source: Sglang Sparse Flash Attention (sparse_attn_func).  Row r of
+ * q-block i of head h attends the keys of blocks [off, off + block_N) for
+ * the first block_count entries of block_offset, plus the first
+ * column_count keys of column_index, with the causal mask if asked.
+ * Index arrays as produced by sbfa_convert_vertical_slash (per query head).
+ * Requires block_M == block_N == 64, Hq == Hkv.
+ */
+sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                                    const int32_t* block_count, const int32_t* block_offset,
+                                    int32_t nnz_s, const int32_t* column_count,
+                                    const int32_t* column_index, int32_t nnz_v,
+                                    int32_t block_M, int32_t block_N, sbfa_t4 o, float* lse,
+                                    int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_check_status -- synchronise `stream`, read the device status word
+ * and map it to SBFA_OK / SBFA_ERR_DEVICE / SBFA_ERR_TIMEOUT.
+ */
+sbfa_status sbfa_check_status(const int32_t* status, sbfa_stream_t stream);
+
+/* Message of the last error on this host thread ("" if none). */
+const char* sbfa_last_error(void);
+
+/* Library version string. */
+const char* sbfa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBFA_H_ */

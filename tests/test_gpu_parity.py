@@ -1,0 +1,272 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.  Tolerances: o max-abs <= 2e-2, lse max-abs <= 1e-3
+(bf16 inputs, fp32 accumulation); integer outputs bit-exact; gate keep bits
+bit-exact except blocks with |s_max - T| < 1e-3, which are reported."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL = 2e-2, 1e-3
+
+
+@pytest.fixture(scope="module")
+def sb():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    import block_sparse_flashattention_sbfa_b200 as m
+    return m
+
+
+def dev(bits):
+    return W.to_torch_bf16(bits, "cuda")
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    """Element-wise comparison on every row the oracle computed."""
+    o = o_gpu.float().cpu().numpy().astype(np.float64)
+    lse = lse_gpu.float().cpu().numpy().astype(np.float64)
+    rows = ~np.isnan(lse_ref)
+    orow = ~np.isnan(o_ref[..., 0])
+    assert orow.sum() > 0
+    err_o = np.abs(o[orow] - o_ref[orow]).max()
+    lr, lg = lse_ref[rows], lse[rows]
+    inf_ref = np.isneginf(lr)
+    assert np.array_equal(inf_ref, np.isneginf(lg)), f"{what}: -inf pattern of lse differs"
+    err_l = np.abs(lg[~inf_ref] - lr[~inf_ref]).max() if (~inf_ref).any() else 0.0
+    print(f"{what}: o max-abs {err_o:.3e}, lse max-abs {err_l:.3e}, rows {rows.sum()}")
+    assert err_o <= O_TOL, f"{what}: o max-abs {err_o}"
+    assert err_l <= LSE_TOL, f"{what}: lse max-abs {err_l}"
+
+
+def sampled_rows(n_rows, block, seed, n=4):
+    rng = np.random.default_rng(seed)
+    nqb = -(-n_rows // block)
+    qbs = W.sample_qblocks(rng, nqb, n)
+    return np.concatenate([np.arange(b * block, min((b + 1) * block, n_rows)) for b in qbs])
+
+
+# ------------------------------------------------------------------ block table
+
+def test_block_table_tiny_workload(sb):
+    """B=1, H=2, Lq=256, Lk=1024, bs=64, non-causal, diagonal + 7 random blocks;
+    plus the LSE combine of the two disjoint halves of every table row."""
+    wl = W.make_block_table()
+    tab = wl.meta["table"]
+    q, k, v = dev(wl.q), dev(wl.k), dev(wl.v)
+    t = torch.from_numpy(tab).cuda()
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd(q, k, v, t, 64, 64, causal=False, status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_block_table(wl.q, wl.k, wl.v, tab, 64, 64, False, wl.scale)
+    compare(o, lse, ro, rl, "block table")
+    # halves -> combine
+    oa, la = sb.fwd(q, k, v, t[..., :4], 64, 64)
+    ob, lb = sb.fwd(q, k, v, t[..., 4:], 64, 64)
+    oc, lc = sb.combine(torch.stack([oa.float(), ob.float()]), torch.stack([la, lb]))
+    compare(oc, lc, ro, rl, "combine of halves")
+    # per-entry partials -> combine
+    op, lp = sb.fwd_partials(q, k, v, t, 64, 64)
+    oc2, lc2 = sb.combine(op, lp)
+    compare(oc2, lc2, ro, rl, "combine of 8 partials")
+    ro0, rl0 = oracle.attend_block_table(wl.q, wl.k, wl.v, tab[..., 3:4], 64, 64, False, wl.scale)
+    compare(op[3], lp[3], ro0, rl0, "partial 3")
+
+
+@pytest.mark.parametrize("G,causal,q_block,kv_block", [(1, True, 64, 64), (2, True, 128, 128),
+                                                        (4, False, 64, 256), (8, True, 192, 64)])
+def test_block_table_ragged_gqa(sb, G, causal, q_block, kv_block):
+    rng = np.random.default_rng(100 + G)
+    B, Sq, Sk, Hkv = 2, 333, 1000, 2
+    Hq = Hkv * G
+    q = W.normal_bf16(rng, (B, Sq, Hq, 128))
+    k = W.normal_bf16(rng, (B, Sk, Hkv, 128))
+    v = W.normal_bf16(rng, (B, Sk, Hkv, 128))
+    nqb, nkb = -(-Sq // q_block), -(-Sk // kv_block)
+    tab = rng.integers(-1, nkb, size=(B, Hkv, nqb, 6)).astype(np.int32)
+    tab[..., 5] = tab[..., 0]                # duplicate entry counts once
+    tab[0, 0, 0, :] = -1                     # an empty row: o = 0, lse = -inf
+    o, lse = sb.fwd(dev(q), dev(k), dev(v), torch.from_numpy(tab).cuda(), q_block, kv_block,
+                    causal=causal)
+    ro, rl = oracle.attend_block_table(q, k, v, tab, q_block, kv_block, causal, W.default_scale())
+    compare(o, lse, ro, rl, f"ragged G={G}")
+
+
+def test_block_table_1d_broadcast_and_dense(sb):
+    rng = np.random.default_rng(7)
+    B, S, H = 1, 512, 4
+    q, k, v = (W.normal_bf16(rng, (B, S, H, 128)) for _ in range(3))
+    full = torch.arange(S // 64, dtype=torch.int32, device="cuda")
+    o1, l1 = sb.fwd(dev(q), dev(k), dev(v), full, 64, 64, causal=True)
+    o2, l2 = sb.fwd_dense(dev(q), dev(k), dev(v), causal=True)
+    tab = np.broadcast_to(np.arange(S // 64, dtype=np.int32), (B, H, 1, S // 64))
+    ro, rl = oracle.attend_block_table(q, k, v, tab, S, 64, True, W.default_scale())
+    compare(o1, l1, ro, rl, "1-D table")
+    compare(o2, l2, ro, rl, "dense")
+
+
+# ------------------------------------------------------------------ decode
+
+def _spec_case(B, Hq, Hkv, Sq, Lk, bs, spec, n_missed, seed):
+    wl = W.make_spec_decode(B=B, Hq=Hq, Hkv=Hkv, Lq=Sq, Lk=Lk, block=bs, spec_len=spec,
+                            n_missed=n_missed, seed=seed, table_seed=seed + 1000)
+    return wl
+
+
+@pytest.mark.parametrize("Sq,causal_spec", [(1, True), (2, True), (4, False)])
+def test_speculative_sparse_small(sb, Sq, causal_spec):
+    wl = _spec_case(2, 8, 2, Sq, 4096, 128, 512, 6, 20 + Sq)
+    t = wl.meta["table"]
+    s0 = wl.meta["spec_begin"]
+    q, k, v = dev(wl.q), dev(wl.k), dev(wl.v)
+    tab = torch.from_numpy(t).cuda()
+    st = sb.new_status("cuda")
+    o, lse = sb.speculative_sparse(q, k[:, s0:], v[:, s0:], causal_spec, k, v, tab, 128,
+                                   status=st)
+    sb.check_status(st)
+    ro, rl = oracle.speculative_sparse(wl.q, wl.k[:, s0:], wl.v[:, s0:], causal_spec, wl.k,
+                                       wl.v, t, 128, wl.scale)
+    compare(o, lse, ro, rl, f"spec fused Sq={Sq}")
+    # three-call path: dense pass A, sparse pass B, combine
+    oa, la = sb.fwd_dense(q, k[:, s0:], v[:, s0:], causal=causal_spec)
+    ob, lb = sb.fwd(q, k, v, tab, max(Sq, 1), 128, causal=False)
+    oc, lc = sb.combine(torch.stack([oa.float(), ob.float()]), torch.stack([la, lb]))
+    compare(oc, lc, ro, rl, f"spec 3-call Sq={Sq}")
+
+
+def test_speculative_sparse_full_workload(sb):
+    """B=8, Hq=32, Hkv=8, Lk=32768, bs=128: dense last 2048 + 32 missed blocks;
+    every (b, h) row checked against attention over the union."""
+    wl = W.make_spec_decode()
+    t = wl.meta["table"]
+    s0 = wl.meta["spec_begin"]
+    q, k, v = dev(wl.q), dev(wl.k), dev(wl.v)
+    tab = torch.from_numpy(t).cuda()
+    ws = sb.decode_workspace(8, 8, 1, 32, "cuda")
+    for rep in range(2):       # the workspace's counters must come back to zero
+        o, lse = sb.speculative_sparse(q, k[:, s0:], v[:, s0:], True, k, v, tab, 128, ws=ws)
+    torch.cuda.synchronize()
+    union = np.concatenate([t, np.broadcast_to(np.arange(s0 // 128, 256, dtype=np.int32),
+                                               (8, 8, 1, 16))], axis=-1)
+    ro, rl = oracle.attend_block_table(wl.q, wl.k, wl.v, union, 1, 128, False, wl.scale)
+    compare(o, lse, ro, rl, "spec decode full")
+
+
+# ------------------------------------------------------------------ gated
+
+def _gated_small(L=1024, Hq=8, Hkv=2, k_top=4):
+    wl = W.make_gated(B=1, Hq=Hq, Hkv=Hkv, L=L, seed=30)
+    cal = W.make_gated(B=1, Hq=Hq, Hkv=Hkv, L=L, seed=31)
+    G = Hq // Hkv
+    sm = np.stack([oracle.block_max_head(cal.q[0, :, h], cal.k[0, :, h // G], 64, cal.scale)
+                   for h in range(Hq)])
+    T = oracle.calibrate_thresholds(sm, k_top).astype(np.float32)
+    return wl, T
+
+
+def _check_keep(info, smax_g, keep_g, T, what):
+    """Keep bits bit-exact except blocks whose s_max is within 1e-3 of T."""
+    n_diff = n_near = n_tot = 0
+    max_sm_err = 0.0
+    for (b, h, i), (sm_ref, keep_ref) in info.items():
+        kg = keep_g[b, h, i, :i + 1].astype(bool)
+        sg = smax_g[b, h, i, :i + 1]
+        max_sm_err = max(max_sm_err, np.abs(sg - sm_ref).max())
+        near = np.abs(sm_ref - T[h, i]) < 1e-3
+        diff = kg != keep_ref
+        n_near += int((diff & near).sum())
+        n_diff += int((diff & ~near).sum())
+        n_tot += i + 1
+    print(f"{what}: {n_tot} blocks, keep mismatches {n_diff}, near-threshold flips {n_near}, "
+          f"s_max max-abs {max_sm_err:.2e}")
+    assert n_diff == 0
+    assert max_sm_err < 1e-3
+    return n_near
+
+
+def test_gated_small_all_rows(sb):
+    wl, T = _gated_small()
+    q, k, v = dev(wl.q), dev(wl.k), dev(wl.v)
+    n = T.shape[1]
+    smax = torch.full((1, 8, n, n), float("nan"), device="cuda")
+    keep = torch.full((1, 8, n, n), 255, dtype=torch.uint8, device="cuda")
+    o, lse = sb.fwd_gated(q, k, v, torch.from_numpy(T).cuda(), smax_out=smax, keep_out=keep)
+    ro, rl, info = oracle.attend_gated(wl.q, wl.k, wl.v, T, 64, wl.scale, return_keep=True)
+    near = _check_keep(info, smax.cpu().numpy(), keep.cpu().numpy(), T, "gated small")
+    if near == 0:
+        compare(o, lse, ro, rl, "gated small")
+    kept = keep.cpu().numpy()
+    assert np.all(kept[0][:, np.triu_indices(n, 1)[0], np.triu_indices(n, 1)[1]] == 255)
+
+
+def test_gated_full_workload_sampled(sb):
+    """Llama-3.1-8B shape, L=32768, 64x64 tiles, T from the stored seed-101
+    calibration; 4 whole q-blocks (256 rows) per head checked."""
+    import os
+    T = np.load(os.path.join(os.path.dirname(__file__), "golden", "gated_T_seed101.npy"))
+    wl = W.make_gated()
+    q, k, v = dev(wl.q), dev(wl.k), dev(wl.v)
+    n = 512
+    smax = torch.empty((1, 32, n, n), device="cuda")
+    keep = torch.empty((1, 32, n, n), dtype=torch.uint8, device="cuda")
+    o, lse = sb.fwd_gated(q, k, v, torch.from_numpy(T).cuda(), smax_out=smax, keep_out=keep)
+    torch.cuda.synchronize()
+    rows = {h: sampled_rows(32768, 64, 500 + h) for h in range(32)}
+    ro, rl, info = oracle.attend_gated(wl.q, wl.k, wl.v, T, 64, wl.scale,
+                                       rows=lambda b, h: rows[h], return_keep=True)
+    kp = keep.cpu().numpy()
+    near = _check_keep(info, smax.cpu().numpy(), kp, T, "gated full")
+    dens = sum(int(kp[0, h, i, :i + 1].sum()) for (_, h, i) in info) / \
+        sum(i + 1 for (_, _, i) in info)
+    print(f"gated full: kept density on the sampled q-blocks {dens:.3f}")
+    if near == 0:
+        compare(o, lse, ro, rl, "gated full")
+
+
+# ------------------------------------------------------------------ vertical-slash
+
+def _vs_small(L=2048, H=4, nnz_v=64, nnz_s=160, seed=40):
+    return W.make_vertical_slash(B=1, H=H, L=L, nnz_v=nnz_v, nnz_s=nnz_s, seed=seed,
+                                 table_seed=seed + 1000)
+
+
+def test_vertical_slash_small(sb):
+    wl = _vs_small()
+    L, H = wl.q.shape[1], wl.q.shape[2]
+    vert, slash = wl.meta["vertical"], wl.meta["slash"]
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    bc, bo, cc, ci = sb.convert_vertical_slash(sl, sl, torch.from_numpy(vert).cuda(),
+                                               torch.from_numpy(slash).cuda(), L)
+    rbc, rbo, rcc, rci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    bc, bo, cc, ci = (x.cpu().numpy() for x in (bc, bo, cc, ci))
+    assert np.array_equal(bc, rbc) and np.array_equal(cc, rcc)
+    for idx in np.ndindex(bc.shape):
+        assert np.array_equal(bo[idx][:bc[idx]], rbo[idx][:rbc[idx]])
+        assert np.array_equal(ci[idx][:cc[idx]], rci[idx][:rcc[idx]])
+    print(f"vs small: mean blocks {bc.mean():.1f}, mean columns {cc.mean():.2f}")
+    o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), *(torch.from_numpy(x).cuda()
+                                   for x in (rbc, rbo, rcc, rci)), causal=True)
+    ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, rbc, rbo, rcc, rci, 64, 64, True,
+                                          wl.scale)
+    compare(o, lse, ro, rl, "vs small")
+
+
+def test_vertical_slash_columns_heavy(sb):
+    """Few slash lines, many vertical columns: most keys come from the column
+    gather path."""
+    wl = _vs_small(L=1536, H=2, nnz_v=400, nnz_s=64, seed=41)
+    L = wl.q.shape[1]
+    vert, slash = wl.meta["vertical"], wl.meta["slash"]
+    rbc, rbo, rcc, rci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    assert rcc.max() > 64
+    o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), *(torch.from_numpy(x).cuda()
+                                   for x in (rbc, rbo, rcc, rci)), causal=True)
+    ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, rbc, rbo, rcc, rci, 64, 64, True,
+                                          wl.scale)
+    compare(o, lse, ro, rl, "vs columns")
