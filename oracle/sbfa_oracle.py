@@ -222,10 +222,12 @@ def speculative_sparse(q, k_spec, v_spec, causal_spec, k, v, table, kv_block, sc
 # ----------------------------------------------------------------------------
 
 def block_max_head(qh, kh, block, scale, i_list=None):
-    """s_max[i, j] = max over rows of q-block i and keys of k-block j of
-    scale * q.k, for one head: qh (L, D), kh (L, D).  Only causal candidates
-    j <= i are evaluated; the rest are -inf.  (BSFA, Figure 2a: per-block
-    maxima computed exactly inside the attention tile.)"""
+    """s_max[i, j] = max over rows r of q-block i and keys c of k-block j of
+    scale * q_r.k_c, for one head: qh (L, D), kh (L, D), causal (c <= r).
+    Only candidates j <= i are evaluated; the rest are -inf.  (BSFA, Figure
+    2a: per-block maxima computed exactly inside the attention tile, where
+    the causal mask hides c > r; this only matters on the diagonal block,
+    which is always kept.)"""
     qh, kh = _f64(qh), _f64(kh)
     L = qh.shape[0]
     n = -(-L // block)
@@ -235,6 +237,7 @@ def block_max_head(qh, kh, block, scale, i_list=None):
         r0, r1 = i * block, min((i + 1) * block, L)
         kend = min((i + 1) * block, L)
         s = scale * (qh[r0:r1] @ kh[:kend].T)          # (rows, keys <= end of block i)
+        s = np.where(np.arange(kend)[None, :] <= np.arange(r0, r1)[:, None], s, NEG_INF)
         pad = (i + 1) * block - kend                   # ragged last key block
         if pad:
             s = np.concatenate([s, np.full((s.shape[0], pad), NEG_INF)], axis=1)
