@@ -1,0 +1,421 @@
+// NSA selected attention over varlen-packed sequences (Flash-Sparse-Attention
+// Quickstart: per-token top-k key blocks of 64, cu_seqlens packing), computed
+// block-major as in FSA's loop-order swap: instead of each query token
+// walking its own top-k blocks (one query row per kv-head: no tensor-core
+// tile), every selected key block gathers the query rows that chose it.
+//
+//   1. nsa_count_kernel / nsa_scan_kernel / nsa_fill_kernel build the
+//      inverted index: for each (kv-head g, block) the list of (token, slot)
+//      pairs that selected it (counting sort).
+//   2. nsa_main_kernel: one unit = one key block and up to 128 query rows
+//      (entries x G query heads) that selected it.  Q rows are gathered with
+//      cp.async into a 128B-swizzled tile, K/V come by TMA, S = Q K^T and
+//      O = P V run on tcgen05 with fp32 accumulators in TMEM.  Each row's
+//      result over that one block is an fp32 partial (o, lse) stored at its
+//      (token, head, slot).
+//   3. nsa_combine_kernel merges the top-k partials of every (token, head)
+//      with the LSE combine.
+#pragma once
+
+#include "sbfa_ptx.cuh"
+
+namespace sbfa {
+
+struct NsaParams {
+  int nseq, total, Hq, Hkv, G, topk, nbps;  // nbps: 64-key blocks per sequence slot
+  int causal;
+  float scale_log2;
+  const int* cu;       // [nseq + 1]
+  const int* sel;      // [total, Hkv, topk]
+  const __nv_bfloat16* q;
+  int64_t qss, qsh;
+  int* count;          // [Hkv * NB]
+  int* cursor;         // [Hkv * NB]
+  int* offset;         // [Hkv * NB + 1]
+  int* unit_prefix;    // [Hkv * NB + 1]
+  int* list;           // [entries]
+  float* part_o;       // [total * Hq * topk, 128]
+  float* part_lse;     // [total * Hq * topk]
+  __nv_bfloat16* o;
+  int64_t oss, osh;
+  float* lse;          // [Hq, total]
+  int* status;
+};
+
+__device__ __forceinline__ int nsa_seq_of(const int* cu, int nseq, int t) {
+  int lo = 0, hi = nseq;  // cu[lo] <= t < cu[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(cu + mid) <= t) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Validate one selection entry; returns the global block id or -1.
+__device__ __forceinline__ int nsa_block_id(const NsaParams& p, int s, int j) {
+  if (j < 0) return -1;
+  const int L = __ldg(p.cu + s + 1) - __ldg(p.cu + s);
+  if (j >= (L + 63) / 64) {
+    report(p.status, kDevBadIndex);
+    return -1;
+  }
+  return s * p.nbps + j;
+}
+
+__global__ void nsa_count_kernel(NsaParams p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(p.total) * p.Hkv * p.topk;
+  if (i >= n) return;
+  const int t = static_cast<int>(i / (p.Hkv * p.topk));
+  const int g = static_cast<int>((i / p.topk) % p.Hkv);
+  const int s = nsa_seq_of(p.cu, p.nseq, t);
+  const int gb = nsa_block_id(p, s, p.sel[i]);
+  if (gb >= 0) atomicAdd(&p.count[g * p.nseq * p.nbps + gb], 1);
+}
+
+// Single CTA: exclusive prefix sums of counts and of units per (g, block).
+__global__ void nsa_scan_kernel(NsaParams p) {
+  __shared__ int warp_tot[2][32];
+  const int n = p.Hkv * p.nseq * p.nbps;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  const int per_unit = 128 / p.G;
+  int carry_e = 0, carry_u = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const int c = i < n ? p.count[i] : 0;
+    const int u = (c + per_unit - 1) / per_unit;
+    int xe = c, xu = u;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int ye = __shfl_up_sync(0xffffffffu, xe, off);
+      const int yu = __shfl_up_sync(0xffffffffu, xu, off);
+      if (lane >= off) { xe += ye; xu += yu; }
+    }
+    if (lane == 31) { warp_tot[0][warp] = xe; warp_tot[1][warp] = xu; }
+    __syncthreads();
+    int be = 0, bu = 0, te = 0, tu = 0;
+    for (int w = 0; w < nw; ++w) {
+      if (w < warp) { be += warp_tot[0][w]; bu += warp_tot[1][w]; }
+      te += warp_tot[0][w];
+      tu += warp_tot[1][w];
+    }
+    if (i < n) {
+      p.offset[i] = carry_e + be + xe - c;
+      p.unit_prefix[i] = carry_u + bu + xu - u;
+      p.cursor[i] = 0;
+    }
+    carry_e += te;
+    carry_u += tu;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    p.offset[n] = carry_e;
+    p.unit_prefix[n] = carry_u;
+  }
+}
+
+__global__ void nsa_fill_kernel(NsaParams p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(p.total) * p.Hkv * p.topk;
+  if (i >= n) return;
+  const int t = static_cast<int>(i / (p.Hkv * p.topk));
+  const int g = static_cast<int>((i / p.topk) % p.Hkv);
+  const int slot = static_cast<int>(i % p.topk);
+  const int s = nsa_seq_of(p.cu, p.nseq, t);
+  const int j = p.sel[i];
+  if (j < 0) return;
+  const int L = p.cu[s + 1] - p.cu[s];
+  if (j >= (L + 63) / 64) return;  // reported by the count pass
+  const int key = g * p.nseq * p.nbps + s * p.nbps + j;
+  const int pos = p.offset[key] + atomicAdd(&p.cursor[key], 1);
+  p.list[pos] = t * p.topk + slot;
+}
+
+// ----------------------------------------------------------------------------
+// main kernel
+// ----------------------------------------------------------------------------
+constexpr int kNsaThreads = 384;
+
+struct NsaSmem {
+  alignas(1024) uint8_t q[2][kQTileBytes];
+  alignas(1024) uint8_t k[2][kTileBytes];
+  alignas(1024) uint8_t v[2][kTileBytes];
+  alignas(1024) uint8_t p[2][kPTileBytes];
+  uint32_t tmem_base;
+  int abort_flag;
+  uint64_t kv_full[2], q_full[2], buf_empty[2];
+  uint64_t s_full[2], p_full[2], o_full[2];
+};
+
+struct NsaUnit {
+  int g, s, j, e0, ne;  // kv head, sequence, local block, first list entry, entries
+};
+
+__device__ __forceinline__ NsaUnit nsa_unit(const NsaParams& p, int u) {
+  const int n = p.Hkv * p.nseq * p.nbps;
+  int lo = 0, hi = n;  // unit_prefix[lo] <= u < unit_prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(p.unit_prefix + mid) <= u) lo = mid; else hi = mid;
+  }
+  // skip (g, block) pairs with no unit (equal prefixes)
+  while (lo + 1 < n && __ldg(p.unit_prefix + lo + 1) <= u) ++lo;
+  NsaUnit r;
+  r.g = lo / (p.nseq * p.nbps);
+  const int gb = lo % (p.nseq * p.nbps);
+  r.s = gb / p.nbps;
+  r.j = gb % p.nbps;
+  const int per_unit = 128 / p.G;
+  const int chunk = u - __ldg(p.unit_prefix + lo);
+  const int cnt = __ldg(p.offset + lo + 1) - __ldg(p.offset + lo);
+  r.e0 = __ldg(p.offset + lo) + chunk * per_unit;
+  r.ne = min(per_unit, cnt - chunk * per_unit);
+  return r;
+}
+
+__global__ void __launch_bounds__(kNsaThreads, 1)
+    nsa_main_kernel(const __grid_constant__ CUtensorMap mapK,
+                    const __grid_constant__ CUtensorMap mapV, const NsaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  NsaSmem& sm = *reinterpret_cast<NsaSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_units = __ldg(p.unit_prefix + p.Hkv * p.nseq * p.nbps);
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.kv_full[b], 1);
+      mbar_init(&sm.q_full[b], 2);
+      mbar_init(&sm.buf_empty[b], 128);
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.p_full[b], 128);
+      mbar_init(&sm.o_full[b], 1);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wctx{&sm.abort_flag, p.status};
+
+  if (warp == 0 || warp == 3) {
+    // ===================== producers: K/V by TMA, Q rows by cp.async =====================
+    const int half = warp == 0 ? 0 : 1;  // rows [64*half, 64*half + 64)
+    int n = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
+      const int b = n & 1;
+      if (lane == 0) ok = mbar_wait(&sm.buf_empty[b], ((n >> 1) & 1) ^ 1u, wctx);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      const NsaUnit un = nsa_unit(p, u);
+      if (half == 0 && lane == 0) {
+        const int key0 = __ldg(p.cu + un.s) + un.j * 64;
+        mbar_arrive_expect_tx(&sm.kv_full[b], 2 * kTileBytes);
+        tma_load_4d(sm.k[b], &mapK, &sm.kv_full[b], 0, un.g, key0, 0);
+        tma_load_4d(sm.k[b] + 8192, &mapK, &sm.kv_full[b], 64, un.g, key0, 0);
+        tma_load_4d(sm.v[b], &mapV, &sm.kv_full[b], 0, un.g, key0, 0);
+        tma_load_4d(sm.v[b] + 8192, &mapV, &sm.kv_full[b], 64, un.g, key0, 0);
+      }
+      const uint32_t d0 = smem_u32(sm.q[b]);
+      for (int e = lane; e < 64 * 16; e += 32) {
+        const int r = half * 64 + (e >> 4), ch = e & 15;
+        const uint32_t saddr = d0 + (ch >> 3) * 16384 + sw128_off(r, ch & 7);
+        const int ent = r / p.G;
+        if (ent < un.ne) {
+          const int code = __ldg(p.list + un.e0 + ent);
+          const int t = code / p.topk;
+          const int h = un.g * p.G + r % p.G;
+          const __nv_bfloat16* src = p.q + static_cast<int64_t>(t) * p.qss + h * p.qsh + ch * 8;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(src)
+                       : "memory");
+        } else {
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(saddr), "r"(0)
+                       : "memory");
+        }
+      }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full[b]);
+    }
+  } else if (warp == 1) {
+    // ===================== MMA issuer =====================
+    // Order: QK(0), QK(1), PV(0), QK(2), PV(1), ... so that the softmax of
+    // one unit overlaps the QK of the next.
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16(128, 64, 0);
+      const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
+      bool ok = true;
+      auto issue_qk = [&](int n) -> bool {
+        const int b = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        if (!mbar_wait(&sm.q_full[b], ph, wctx) || !mbar_wait(&sm.kv_full[b], ph, wctx))
+          return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sm.q[b]), ka = smem_u32(sm.k[b]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          umma_ss(tmem + b * 256, ad, bd, idesc_qk, kk ? 1u : 0u);
+        }
+        umma_commit(&sm.s_full[b]);
+        return true;
+      };
+      auto issue_pv = [&](int n) -> bool {
+        const int b = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        if (!mbar_wait(&sm.p_full[b], ph, wctx)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sm.p[b]), va = smem_u32(sm.v[b]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = sdesc_sw128(pa + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(va + kk * 2048, 8192, 1024);
+          umma_ss(tmem + b * 256 + 128, ad, bd, idesc_pv, kk ? 1u : 0u);
+        }
+        umma_commit(&sm.o_full[b]);
+        return true;
+      };
+      int n_mine = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) ++n_mine;
+      if (n_mine > 0) ok = issue_qk(0);
+      for (int n = 0; n < n_mine && ok; ++n) {
+        if (n + 1 < n_mine) ok = issue_qk(n + 1);
+        if (ok) ok = issue_pv(n);
+      }
+      // drain every tcgen05 op before TMEM is released
+      umma_commit(&sm.s_full[0]);
+      mbar_wait_short(&sm.s_full[0], ((n_mine + 1) >> 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ===================== softmax / epilogue warpgroups (ping-pong) =====================
+    const int b = (warp - 4) >> 2;
+    const int r = tid - 128 - 128 * b;
+    const int quarter = warp & 3;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * 256;
+    const float NEG = -INFINITY;
+    int n = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
+      if ((n & 1) != b) continue;
+      const uint32_t ph = (n >> 1) & 1;
+      const NsaUnit un = nsa_unit(p, u);
+      const int ent = r / p.G;
+      const bool valid = ent < un.ne;
+      int t = 0, slot = 0, tl = 0, L = 0;
+      if (valid) {
+        const int code = __ldg(p.list + un.e0 + ent);
+        t = code / p.topk;
+        slot = code % p.topk;
+        const int base = __ldg(p.cu + un.s);
+        tl = t - base;
+        L = __ldg(p.cu + un.s + 1) - base;
+      }
+      if (!mbar_wait(&sm.s_full[b], ph, wctx)) { ok = false; break; }
+      tc_fence_after();
+      float s[64];
+      tmem_ld32(lane_addr, s);
+      tmem_ld32(lane_addr + 32, s + 32);
+      float mx = NEG;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int key = un.j * 64 + c;
+        const bool vis = valid && key < L && (!p.causal || key <= tl);
+        s[c] = vis ? s[c] * p.scale_log2 : NEG;
+        mx = fmaxf(mx, s[c]);
+      }
+      const float mu = (mx == NEG) ? 0.f : mx;
+      float l = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = ex2_approx(s[c] - mu), p1 = ex2_approx(s[c + 1] - mu);
+        l += p0 + p1;
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+      }
+      const uint32_t prow = smem_u32(sm.p[b]);
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, cc)),
+                     "r"(pk[cc * 4]), "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
+                     : "memory");
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[b]);
+      if (!mbar_wait(&sm.o_full[b], ph, wctx)) { ok = false; break; }
+      tc_fence_after();
+      const int h = un.g * p.G + r % p.G;
+      const int64_t prow_idx = (static_cast<int64_t>(t) * p.Hq + h) * p.topk + slot;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float ob[32];
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(lane_addr + 128 + c * 32, ob);
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + prow_idx * 128 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(ob[4 * i] * inv, ob[4 * i + 1] * inv, ob[4 * i + 2] * inv,
+                                 ob[4 * i + 3] * inv);
+        }
+      }
+      if (valid) p.part_lse[prow_idx] = l > 0.f ? (mu + lg2_approx(l)) * 0.69314718055994531f : NEG;
+      tc_fence_before();
+      mbar_arrive(&sm.buf_empty[b]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// One warp per (token, query head): LSE combine of its valid slots.
+__global__ void nsa_combine_kernel(NsaParams p) {
+  const int64_t wg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wg >= static_cast<int64_t>(p.total) * p.Hq) return;
+  const int t = static_cast<int>(wg / p.Hq), h = static_cast<int>(wg % p.Hq);
+  const int g = h / p.G;
+  const int s = nsa_seq_of(p.cu, p.nseq, t);
+  const int L = p.cu[s + 1] - p.cu[s];
+  const int nb = (L + 63) / 64;
+  const int* sl = p.sel + (static_cast<int64_t>(t) * p.Hkv + g) * p.topk;
+  const int64_t row = (static_cast<int64_t>(t) * p.Hq + h) * p.topk;
+  float M = -INFINITY;
+  for (int k = 0; k < p.topk; ++k) {
+    const int j = __ldg(sl + k);
+    if (j < 0 || j >= nb) continue;
+    M = fmaxf(M, p.part_lse[row + k]);
+  }
+  const float Mn = (M == -INFINITY) ? 0.f : M;
+  float W = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < p.topk; ++k) {
+    const int j = __ldg(sl + k);
+    if (j < 0 || j >= nb) continue;
+    const float lv = p.part_lse[row + k];
+    if (lv == -INFINITY) continue;
+    const float w = __expf(lv - Mn);
+    W += w;
+    const float4 x = *reinterpret_cast<const float4*>(p.part_o + (row + k) * 128 + lane * 4);
+    acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  __nv_bfloat16* op = p.o + static_cast<int64_t>(t) * p.oss + h * p.osh + lane * 4;
+  reinterpret_cast<__nv_bfloat162*>(op)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  reinterpret_cast<__nv_bfloat162*>(op)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  if (lane == 0) p.lse[static_cast<int64_t>(h) * p.total + t] = W > 0.f ? Mn + __logf(W) : -INFINITY;
+}
+
+}  // namespace sbfa

@@ -14,6 +14,7 @@
 #include "kernel_convert.cuh"
 #include "kernel_decode.cuh"
 #include "kernel_prefill.cuh"
+#include "kernel_nsa.cuh"
 
 namespace {
 
@@ -309,6 +310,30 @@ sbfa_status check_table(const sbfa_table* t, const sbfa_shape* s, bool prefill) 
   return SBFA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// NSA selected attention workspace
+// ---------------------------------------------------------------------------
+struct NsaWs {
+  size_t count, cursor, offset, unit_prefix, list, part_lse, part_o, total;
+};
+
+size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+NsaWs nsa_ws_layout(int nseq, int total, int max_seqlen, int Hq, int Hkv, int topk) {
+  const size_t nb = static_cast<size_t>(Hkv) * nseq * ((max_seqlen + 63) / 64);
+  NsaWs w;
+  size_t off = 0;
+  w.count = off; off += al256(nb * 4);
+  w.cursor = off; off += al256(nb * 4);
+  w.offset = off; off += al256((nb + 1) * 4);
+  w.unit_prefix = off; off += al256((nb + 1) * 4);
+  w.list = off; off += al256(static_cast<size_t>(total) * Hkv * topk * 4);
+  w.part_lse = off; off += al256(static_cast<size_t>(total) * Hq * topk * 4);
+  w.part_o = off; off += al256(static_cast<size_t>(total) * Hq * topk * 128 * 4);
+  w.total = off;
+  return w;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -536,6 +561,88 @@ sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
   p.vs_nqb = (shape->Sq + 63) / 64;
   p.status = status;
   return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sbfa_varlen_selected_workspace_size(int32_t nseq, int32_t total, int32_t max_seqlen,
+                                           int32_t Hq, int32_t Hkv, int32_t topk) {
+  if (nseq <= 0 || total <= 0 || max_seqlen <= 0 || Hq <= 0 || Hkv <= 0 || topk <= 0) return 0;
+  return nsa_ws_layout(nseq, total, max_seqlen, Hq, Hkv, topk).total;
+}
+
+sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, int32_t total,
+                                     int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                     float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k,
+                                     sbfa_t4 v, const int32_t* sel, int32_t topk, int32_t block,
+                                     void* ws, size_t ws_bytes, sbfa_t4 o, float* lse,
+                                     int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  if (!cu_seqlens || !sel || !ws || !lse) return fail(SBFA_ERR_INVALID_ARG, "null pointer");
+  if (nseq <= 0 || total <= 0 || max_seqlen <= 0 || Hq <= 0 || Hkv <= 0 || topk <= 0)
+    return fail(SBFA_ERR_INVALID_ARG, "non-positive size");
+  if (D != 128) return fail(SBFA_ERR_UNSUPPORTED, "head dim %d (only 128)", D);
+  if (block != 64) return fail(SBFA_ERR_UNSUPPORTED, "selection block %d (only 64)", block);
+  if (Hq % Hkv || 128 % (Hq / Hkv)) return fail(SBFA_ERR_UNSUPPORTED, "Hq/Hkv must divide 128");
+  if (causal != 0 && causal != 1) return fail(SBFA_ERR_INVALID_ARG, "causal must be 0/1");
+  if (static_cast<int64_t>(total) * topk >= (1ll << 31))
+    return fail(SBFA_ERR_UNSUPPORTED, "total * topk too large");
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_view(o, "o", false));
+  const NsaWs L = nsa_ws_layout(nseq, total, max_seqlen, Hq, Hkv, topk);
+  if (ws_bytes < L.total)
+    return fail(SBFA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  if (!aligned16(ws)) return fail(SBFA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  DevInfo di;
+  SBFA_TRY(dev_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  sbfa::NsaParams p{};
+  p.nseq = nseq; p.total = total; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.topk = topk;
+  p.nbps = (max_seqlen + 63) / 64;
+  p.causal = causal;
+  p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt(128.f)) * 1.4426950408889634f;
+  p.cu = cu_seqlens; p.sel = sel;
+  p.q = static_cast<const __nv_bfloat16*>(q.ptr); p.qss = q.ss; p.qsh = q.sh;
+  p.count = reinterpret_cast<int*>(w + L.count);
+  p.cursor = reinterpret_cast<int*>(w + L.cursor);
+  p.offset = reinterpret_cast<int*>(w + L.offset);
+  p.unit_prefix = reinterpret_cast<int*>(w + L.unit_prefix);
+  p.list = reinterpret_cast<int*>(w + L.list);
+  p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
+  p.part_o = reinterpret_cast<float*>(w + L.part_o);
+  p.o = static_cast<__nv_bfloat16*>(o.ptr); p.oss = o.ss; p.osh = o.sh;
+  p.lse = lse;
+  p.status = status;
+  const int64_t nb = static_cast<int64_t>(Hkv) * nseq * p.nbps;
+  if (nb > (1 << 26)) return fail(SBFA_ERR_UNSUPPORTED, "too many key blocks");
+  CUtensorMap mk, mv;
+  SBFA_TRY(encode_bshd(&mk, k, 1, total, Hkv, 64));
+  SBFA_TRY(encode_bshd(&mv, v, 1, total, Hkv, 64));
+  SBFA_CUDA(cudaMemsetAsync(p.count, 0, nb * 4, st));
+  const int64_t n_sel = static_cast<int64_t>(total) * Hkv * topk;
+  const unsigned g1 = static_cast<unsigned>((n_sel + 255) / 256);
+  sbfa::nsa_count_kernel<<<g1, 256, 0, st>>>(p);
+  SBFA_CUDA(cudaGetLastError());
+  sbfa::nsa_scan_kernel<<<1, 1024, 0, st>>>(p);
+  SBFA_CUDA(cudaGetLastError());
+  sbfa::nsa_fill_kernel<<<g1, 256, 0, st>>>(p);
+  SBFA_CUDA(cudaGetLastError());
+  const size_t smem = sizeof(sbfa::NsaSmem) + 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  SBFA_CUDA(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::nsa_main_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr_set[dev] = true;
+  }
+  sbfa::nsa_main_kernel<<<di.sms, sbfa::kNsaThreads, smem, st>>>(mk, mv, p);
+  SBFA_CUDA(cudaGetLastError());
+  const int64_t rows = static_cast<int64_t>(total) * Hq;
+  sbfa::nsa_combine_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
 }
 
 sbfa_status sbfa_check_status(const int32_t* status, sbfa_stream_t stream) {

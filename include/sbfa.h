@@ -211,6 +211,34 @@ sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
                                     int32_t* status, sbfa_stream_t stream);
 
 /*
+ * sbfa_fwd_varlen_selected -- NSA selected attention over varlen sequences.
+ * Source: Flash-Sparse-Attention (FSA), overview and Quickstart (top-k key
+ * blocks of 64 per token, cu_seqlens packing, FSA's block-major loop order).
+ * Token t (sequence-local index tl) of query head h attends the keys of its
+ * selected blocks sel[t, h/G, :] (sequence-local block indices, -1 =
+ * padding, distinct), clipped to its sequence and, if causal, to keys <= tl.
+ * cu_seqlens: int32 [nseq + 1] (device), 0 = cu[0] < ... < cu[nseq] = total;
+ * max_seqlen >= every sequence length.  q: (1, total, Hq, 128) view, k and v:
+ * (1, total, Hkv, 128) views (sb ignored); o like q; lse: fp32 [Hq, total].
+ * sel: int32 [total, Hkv, topk] contiguous.  block must be 64; Hq/Hkv must
+ * divide 128.  ws: device workspace of sbfa_varlen_selected_workspace_size()
+ * bytes (contents need no initialisation).  Runs six launches on `stream`:
+ * inverted-index count / scan / fill, the block-major tcgen05 kernel that
+ * writes one fp32 partial (o, lse) per (token, head, slot), and the LSE
+ * combine of each row's partials.
+ */
+sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, int32_t total,
+                                     int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
+                                     float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k,
+                                     sbfa_t4 v, const int32_t* sel, int32_t topk, int32_t block,
+                                     void* ws, size_t ws_bytes, sbfa_t4 o, float* lse,
+                                     int32_t* status, sbfa_stream_t stream);
+
+/* Workspace bytes for sbfa_fwd_varlen_selected (0 on bad sizes). */
+size_t sbfa_varlen_selected_workspace_size(int32_t nseq, int32_t total, int32_t max_seqlen,
+                                           int32_t Hq, int32_t Hkv, int32_t topk);
+
+/*
  * sbfa_check_status -- synchronise `stream`, read the device status word
  * and map it to SBFA_OK / SBFA_ERR_DEVICE / SBFA_ERR_TIMEOUT.
  */
