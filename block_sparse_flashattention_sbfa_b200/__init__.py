@@ -59,11 +59,15 @@ _SIGS = {
                                     _P, _P, _P],
     "sbfa_fwd_vertical_slash": [ctypes.POINTER(Shape), T4, T4, T4, _P, _P, _I, _P, _P, _I, _I,
                                 _I, T4, _P, _P, _P],
+    "sbfa_fwd_varlen_selected": [_P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, T4, T4, T4, _P,
+                                 _I, _I, _P, ctypes.c_size_t, T4, _P, _P, _P],
+    "sbfa_varlen_selected_workspace_size": [_I, _I, _I, _I, _I, _I],
     "sbfa_check_status": [_P, _P],
     "sbfa_last_error": [],
     "sbfa_version": [],
 }
-_RESTYPES = {"sbfa_decode_workspace_size": ctypes.c_size_t, "sbfa_last_error": ctypes.c_char_p,
+_RESTYPES = {"sbfa_decode_workspace_size": ctypes.c_size_t,
+             "sbfa_varlen_selected_workspace_size": ctypes.c_size_t, "sbfa_last_error": ctypes.c_char_p,
              "sbfa_version": ctypes.c_char_p}
 
 
@@ -71,7 +75,7 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m block_sparse_flashattention_sbfa_b200.build` (nvcc, sm_100a)")
+            "`python block_sparse_flashattention_sbfa_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, args in _SIGS.items():
         fn = getattr(lib, name)
@@ -272,6 +276,37 @@ def fwd_vertical_slash(q, k, v, block_count, block_offset, column_count, column_
           block_count.data_ptr(), block_offset.data_ptr(), block_offset.shape[-1],
           column_count.data_ptr(), column_index.data_ptr(), column_index.shape[-1], block_M,
           block_N, _t4(out), lse.data_ptr(), _ptr(status), _stream())
+    return out, lse
+
+
+def varlen_selected_workspace(nseq, total, max_seqlen, Hq, Hkv, topk, device=None):
+    n = lib.sbfa_varlen_selected_workspace_size(nseq, total, max_seqlen, Hq, Hkv, topk)
+    if n == 0:
+        raise SbfaError("sbfa_varlen_selected_workspace_size", ERR_INVALID_ARG)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def fwd_varlen_selected(q, k, v, cu_seqlens, max_seqlen, sel, block=64, causal=True,
+                        scale=None, ws=None, out=None, lse=None, status=None):
+    """NSA selected attention over varlen-packed sequences
+    (``sbfa_fwd_varlen_selected``).  q (total, Hq, D), k/v (total, Hkv, D),
+    sel int32 (total, Hkv, topk).  Returns o (total, Hq, D), lse (Hq, total)."""
+    _check_bf16(q, k, v)
+    total, Hq, D = q.shape
+    Hkv, topk = k.shape[1], sel.shape[2]
+    nseq = cu_seqlens.numel() - 1
+    if sel.dtype != torch.int32 or not sel.is_contiguous() or cu_seqlens.dtype != torch.int32:
+        raise TypeError("sel and cu_seqlens must be contiguous int32")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, total, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = varlen_selected_workspace(nseq, total, max_seqlen, Hq, Hkv, topk, q.device)
+    _call("sbfa_fwd_varlen_selected", cu_seqlens.data_ptr(), nseq, total, max_seqlen, Hq, Hkv, D,
+          0.0 if scale is None else float(scale), int(bool(causal)), _t4(q[None]), _t4(k[None]),
+          _t4(v[None]), sel.data_ptr(), topk, block, ws.data_ptr(), ws.numel(), _t4(out[None]),
+          lse.data_ptr(), _ptr(status), _stream())
     return out, lse
 
 

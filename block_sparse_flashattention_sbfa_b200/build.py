@@ -1,6 +1,7 @@
 """Compile libsbfa.so (the C-ABI library) for sm_100a, in-tree.
 
-Usage: python -m block_sparse_flashattention_sbfa_b200.build [--verbose-ptxas]
+Usage: python block_sparse_flashattention_sbfa_b200/build.py [--verbose-ptxas]
+(run it as a script: importing the package needs the library it builds).
 """
 import os
 import subprocess

@@ -18,8 +18,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def sb():
-    from block_sparse_flashattention_sbfa_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import block_sparse_flashattention_sbfa_b200 as m
     return m
 

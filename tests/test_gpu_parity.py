@@ -270,3 +270,40 @@ def test_vertical_slash_columns_heavy(sb):
     ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, rbc, rbo, rcc, rci, 64, 64, True,
                                           wl.scale)
     compare(o, lse, ro, rl, "vs columns")
+
+
+# ------------------------------------------------------------------ NSA selected (varlen)
+
+def _nsa_case(seqlens, H, seed):
+    return W.make_nsa_varlen(seqlens=seqlens, H=H, seed=seed, table_seed=seed + 1000)
+
+
+@pytest.mark.parametrize("seqlens", [(700, 300), (1000, 64, 5)])
+def test_nsa_varlen_small_all_tokens(sb, seqlens):
+    wl = _nsa_case(seqlens, 2, 60 + len(seqlens))
+    cu, sel = wl.meta["cu_seqlens"], wl.meta["sel"]
+    q, k, v = (dev(x)[0] for x in (wl.q, wl.k, wl.v))
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_varlen_selected(q, k, v, torch.from_numpy(cu).cuda(), max(seqlens),
+                                    torch.from_numpy(sel).cuda(), status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_selected_varlen(wl.q[0], wl.k[0], wl.v[0], cu, sel, 64, True, wl.scale)
+    compare(o[None], lse[None], ro[None], rl[None], f"nsa small {seqlens}")
+
+
+def test_nsa_varlen_full_workload_sampled(sb):
+    """cu_seqlens [0, 65536, 98304], Hq=Hkv=4, top-16 blocks of 64; 4 whole
+    64-token blocks (256 tokens) per head checked, incl. each sequence's last."""
+    wl = W.make_nsa_varlen()
+    cu, sel = wl.meta["cu_seqlens"], wl.meta["sel"]
+    q, k, v = (dev(x)[0] for x in (wl.q, wl.k, wl.v))
+    ws = sb.varlen_selected_workspace(2, 98304, 65536, 4, 4, 16, "cuda")
+    for _ in range(2):
+        o, lse = sb.fwd_varlen_selected(q, k, v, torch.from_numpy(cu).cuda(), 65536,
+                                        torch.from_numpy(sel).cuda(), ws=ws)
+    torch.cuda.synchronize()
+    rows = {h: np.concatenate([sampled_rows(65536, 64, 700 + h, n=2),
+                               65536 + sampled_rows(32768, 64, 800 + h, n=2)]) for h in range(4)}
+    ro, rl = oracle.attend_selected_varlen(wl.q[0], wl.k[0], wl.v[0], cu, sel, 64, True,
+                                           wl.scale, rows=lambda h: rows[h])
+    compare(o[None], lse[None], ro[None], rl[None], "nsa full")
