@@ -53,6 +53,8 @@ _SIGS = {
     "sbfa_combine": [_I, _I, _I, _I, _I, _P, _P, T4, _P, _P],
     "sbfa_speculative_sparse": [ctypes.POINTER(Shape), T4, T4, T4, _I, _I, T4, T4,
                                 ctypes.POINTER(Table), _P, ctypes.c_size_t, T4, _P, _P, _P],
+    "sbfa_speculative_sparse_noalloc": [ctypes.POINTER(Shape), T4, T4, T4, _I, _I, T4, T4,
+                                        ctypes.POINTER(Table), T4, _P, _P, _P],
     "sbfa_decode_workspace_size": [_I, _I, _I, _I],
     "sbfa_fwd_gated": [ctypes.POINTER(Shape), T4, T4, T4, _P, _I, T4, _P, _P, _P, _P, _P],
     "sbfa_convert_vertical_slash": [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
@@ -225,6 +227,22 @@ def speculative_sparse(q, k_spec, v_spec, causal_spec, k, v, table, kv_block, sc
     _call("sbfa_speculative_sparse", ctypes.byref(shp), _t4(q), _t4(k_spec), _t4(v_spec),
           k_spec.shape[1], int(bool(causal_spec)), _t4(k), _t4(v), ctypes.byref(tb),
           ws.data_ptr(), ws.numel(), _t4(out), lse.data_ptr(), _ptr(status), _stream())
+    return out, lse
+
+
+def speculative_sparse_noalloc(q, k_spec, v_spec, causal_spec, k, v, table, kv_block,
+                               scale=None, out=None, lse=None, status=None):
+    """``sbfa_speculative_sparse_noalloc``: the fused decode with the
+    library's fixed scratch instead of a workspace (for callers that cannot
+    allocate).  Pass preallocated ``out``/``lse`` to allocate nothing here
+    either.  Calls that overlap on the GPU race on the shared scratch."""
+    _check_bf16(q, k_spec, v_spec, k, v)
+    out, lse = _outputs(q, out, lse)
+    tb = _table(table, max(q.shape[1], 1), kv_block)
+    shp = _shape(q, k, False, scale)
+    _call("sbfa_speculative_sparse_noalloc", ctypes.byref(shp), _t4(q), _t4(k_spec),
+          _t4(v_spec), k_spec.shape[1], int(bool(causal_spec)), _t4(k), _t4(v),
+          ctypes.byref(tb), _t4(out), lse.data_ptr(), _ptr(status), _stream())
     return out, lse
 
 

@@ -216,7 +216,7 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
                           const sbfa_t4* kA, const sbfa_t4* vA, int S_A, int causal_A,
                           const sbfa_t4* kB, const sbfa_t4* vB, const sbfa_table* tb, void* ws,
                           size_t ws_bytes, const sbfa_t4& o, float* lse, int32_t* status,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int grid_cap = 0, int ticket_pairs = 0) {
   DevInfo di;
   SBFA_TRY(dev_info(&di));
   const int G = s->Hq / s->Hkv;
@@ -253,14 +253,15 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
   }
   if (!kA) { mKA = mKB; mVA = mVB; }
   if (!tb) { mKB = mKA; mVB = mVA; }
-  const int grid = di.sms;
+  const int grid = (grid_cap > 0 && grid_cap < di.sms) ? grid_cap : di.sms;
   if (ws) {
-    const size_t need = decode_ws_bytes(npairs, grid);
+    const int tpairs = ticket_pairs > npairs ? ticket_pairs : npairs;
+    const size_t need = decode_ws_bytes(tpairs, grid);
     if (ws_bytes < need)
       return fail(SBFA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
     if (!aligned16(ws)) return fail(SBFA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
     uint8_t* w = static_cast<uint8_t*>(ws);
-    const size_t tick = ((static_cast<size_t>(npairs) * 4 + 255) / 256) * 256;
+    const size_t tick = ((static_cast<size_t>(tpairs) * 4 + 255) / 256) * 256;
     p.ws_ticket = reinterpret_cast<int*>(w);
     p.ws_part = reinterpret_cast<float*>(w + tick);
     p.ws_lse = reinterpret_cast<float*>(w + tick +
@@ -332,6 +333,44 @@ NsaWs nsa_ws_layout(int nseq, int total, int max_seqlen, int Hq, int Hkv, int to
   w.part_o = off; off += al256(static_cast<size_t>(total) * Hq * topk * 128 * 4);
   w.total = off;
   return w;
+}
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for sbfa_speculative_sparse_noalloc
+// ---------------------------------------------------------------------------
+// Callers that cannot allocate device memory (code running inside an
+// allocator hook or under a memory budget owned by someone else, or a host
+// with no allocator of its own to call) use this file-scope array instead of
+// a caller-provided workspace.  It holds the split-KV decode kernel's
+// per-pair tickets and per-CTA fp32 partials for up to kNoAllocMaxPairs
+// (batch x kv-head) pairs and kNoAllocMaxCtas CTAs.  Every GPU that loads
+// the library keeps it until the process exits; all calls share it.
+constexpr int kNoAllocMaxPairs = 4096;
+constexpr int kNoAllocMaxCtas = 160;
+constexpr size_t kNoAllocTicketBytes = kNoAllocMaxPairs * 4;
+constexpr size_t kNoAllocBytes =
+    kNoAllocTicketBytes +
+    static_cast<size_t>(kNoAllocMaxCtas) * 2 * sbfa::kDecRows * (sbfa::kDecD + 1) * 4;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch for the current device.  In host code
+// the array's name is only a stand-in, so the address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+sbfa_status noalloc_scratch(void** out) {
+  static void* addr[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  SBFA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(SBFA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return SBFA_OK;
 }
 
 }  // namespace
@@ -479,6 +518,44 @@ sbfa_status sbfa_speculative_sparse(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
   sbfa::DecodeParams p{};
   return launch_decode(p, shape, q, &k_spec, &v_spec, S_spec, causal_spec, &k, &v, missed, ws,
                        ws_bytes, o, lse, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_speculative_sparse_noalloc(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k_spec,
+                                            sbfa_t4 v_spec, int32_t S_spec, int32_t causal_spec,
+                                            sbfa_t4 k, sbfa_t4 v, const sbfa_table* missed,
+                                            sbfa_t4 o, float* lse, int32_t* status,
+                                            sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", false));
+  SBFA_TRY(check_view(k_spec, "k_spec", true));
+  SBFA_TRY(check_view(v_spec, "v_spec", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  if (S_spec <= 0) return fail(SBFA_ERR_INVALID_ARG, "S_spec <= 0");
+  if (causal_spec != 0 && causal_spec != 1) return fail(SBFA_ERR_INVALID_ARG, "causal_spec");
+  if (!decode_shape(shape))
+    return fail(SBFA_ERR_UNSUPPORTED, "Sq * Hq/Hkv = %d > %d", shape->Sq * (shape->Hq / shape->Hkv),
+                sbfa::kDecRows);
+  SBFA_TRY(check_table(missed, shape, false));
+  if (missed->q_block < shape->Sq) return fail(SBFA_ERR_UNSUPPORTED, "missed->q_block < Sq");
+  const int npairs = shape->B * shape->Hkv;
+  if (npairs > kNoAllocMaxPairs)
+    return fail(SBFA_ERR_UNSUPPORTED,
+                "B*Hkv = %d exceeds the fixed scratch limit of %d pairs (use "
+                "sbfa_speculative_sparse with a workspace)", npairs, kNoAllocMaxPairs);
+  void* scratch = nullptr;
+  SBFA_TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the tickets must start at zero (a previous call may have stopped early)
+  SBFA_CUDA(cudaMemsetAsync(scratch, 0, static_cast<size_t>(npairs) * 4, st));
+  // lay the partials out after the full ticket area, as decode_ws_bytes does
+  // for npairs = kNoAllocMaxPairs
+  sbfa::DecodeParams p{};
+  return launch_decode(p, shape, q, &k_spec, &v_spec, S_spec, causal_spec, &k, &v, missed,
+                       scratch, kNoAllocBytes, o, lse, status, st, kNoAllocMaxCtas,
+                       kNoAllocMaxPairs);
 }
 
 sbfa_status sbfa_fwd_gated(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,

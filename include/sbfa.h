@@ -147,6 +147,34 @@ sbfa_status sbfa_speculative_sparse(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
                                     void* ws, size_t ws_bytes, sbfa_t4 o, float* lse,
                                     int32_t* status, sbfa_stream_t stream);
 
+/*
+ * sbfa_speculative_sparse_noalloc -- sbfa_speculative_sparse without a
+ * caller workspace.  The pages have no counterpart: this entry point exists
+ * for callers that cannot call cudaMalloc -- for example code that runs
+ * inside a caching allocator's own callback (allocating there re-enters the
+ * allocator), code whose device memory is a fixed pool owned by another
+ * framework, or latency-critical paths that must not risk the implicit
+ * device synchronisation a cudaMalloc can cause.
+ * Instead of `ws` it uses a fixed scratch array compiled into the library
+ * (about 2.6 MB per GPU that loads the library, held until the process
+ * exits): per-pair tickets and per-CTA fp32 partials for at most 4096
+ * (batch x kv-head) pairs.  Larger B*Hkv is rejected with
+ * SBFA_ERR_UNSUPPORTED.  Allocates nothing: each call zeroes the tickets it
+ * uses with cudaMemsetAsync on `stream`, then launches the same split-KV
+ * kernel.  The first call on a device looks up the scratch array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls share the one array, which keeps
+ * the last call's contents: calls that overlap on the GPU (other streams,
+ * other host threads) race and give wrong results.
+ * Arguments, limits and results are otherwise those of
+ * sbfa_speculative_sparse.
+ */
+sbfa_status sbfa_speculative_sparse_noalloc(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k_spec,
+                                            sbfa_t4 v_spec, int32_t S_spec, int32_t causal_spec,
+                                            sbfa_t4 k, sbfa_t4 v, const sbfa_table* missed,
+                                            sbfa_t4 o, float* lse, int32_t* status,
+                                            sbfa_stream_t stream);
+
 /* Workspace bytes the split-KV decode kernel needs on the current device. */
 size_t sbfa_decode_workspace_size(int32_t B, int32_t Hkv, int32_t Sq, int32_t Hq);
 
