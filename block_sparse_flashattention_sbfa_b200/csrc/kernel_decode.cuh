@@ -22,7 +22,14 @@ namespace sbfa {
 
 constexpr int kDecChunk = 64;
 constexpr int kDecStages = 4;
-constexpr int kDecConsumerWarps = 4;
+constexpr int kDecGroupWarps = 4;                        // warps per consumer group
+constexpr int kDecGroups = 2;                            // groups take alternate chunks
+constexpr int kDecConsumerWarps = kDecGroupWarps * kDecGroups;
+// Chunk k uses stage k % kDecStages and group k % kDecGroups.  The stage count
+// must be a multiple of the group count so that every stage is always
+// consumed by the same group: a group then waits on a stage's phases strictly
+// in order and a parity wait can never be satisfied by an older phase.
+static_assert(kDecStages % kDecGroups == 0, "each stage must belong to one consumer group");
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr int kDecMaxPairs = 4096;
 constexpr int kDecMaxEntries = 1024;
@@ -55,9 +62,9 @@ struct DecStageMeta {
 
 struct DecSmem {
   alignas(1024) uint8_t stage[kDecStages][kDecStageBytes];
-  float mw[kDecConsumerWarps][kDecRows];
-  float lw[kDecConsumerWarps][kDecRows];
-  float ow[kDecConsumerWarps][kDecRows][kDecD];
+  float mw[kDecGroupWarps][kDecRows];
+  float lw[kDecGroupWarps][kDecRows];
+  float ow[kDecGroupWarps][kDecRows][kDecD];
   int prefix[kDecMaxPairs + 1];
   int entries[kDecMaxEntries];
   DecStageMeta meta[kDecStages];
@@ -151,26 +158,37 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kDecConsumerWarps);
+      mbar_init(&sm.empty[s], kDecGroupWarps);
     }
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   // ---- per-pair chunk counts and their prefix sum (every CTA computes the same)
-  for (int pr = tid; pr < npairs; pr += kDecThreads) {
-    int cnt = nA;
-    if (p.has_B) {
-      const int b = pr / p.Hkv, g = pr % p.Hkv;
-      const int* row = p.idx + b * p.tsb + g * p.tsh;
-      int nv = 0;
-      for (int n = 0; n < p.nmax; ++n) {
-        const int j = row[n];
-        if (j >= 0 && j < p.n_kb) ++nv;
-        else if (j >= p.n_kb && cta == 0) report(p.status, kDevBadIndex);
+  // per-pair chunk counts: every thread scans a share of the table entries
+  for (int pr = tid; pr < npairs; pr += kDecThreads) sm.prefix[pr + 1] = nA;
+  __syncthreads();
+  if (p.has_B) {
+    const int n_ent = npairs * p.nmax;
+    for (int base = 0; base < n_ent; base += 4 * kDecThreads) {
+      int jv[4], pv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = base + u * kDecThreads + tid;
+        pv[u] = -1;
+        jv[u] = -1;
+        if (e < n_ent) {
+          const int pr = e / p.nmax, n = e % p.nmax;
+          pv[u] = pr;
+          jv[u] = __ldg(p.idx + (pr / p.Hkv) * p.tsb + (pr % p.Hkv) * p.tsh + n);
+        }
       }
-      cnt += nv * cpe;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (pv[u] < 0) continue;
+        if (jv[u] >= 0 && jv[u] < p.n_kb) atomicAdd(&sm.prefix[pv[u] + 1], cpe);
+        else if (jv[u] >= p.n_kb && cta == 0) report(p.status, kDevBadIndex);
+      }
     }
-    sm.prefix[pr + 1] = cnt;
   }
   __syncthreads();
   if (warp == 0) {
@@ -278,10 +296,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 
   // ======================= consumer warps =======================
+  // Two groups of four warps take alternate chunks; in a chunk warp w of a
+  // group owns keys [16w, 16w + 16).  Per warp: S (16 rows x 16 keys) by
+  // mma.sync with K fragments from ldmatrix, online softmax with a lazily
+  // raised running max, O (16 x 128) += P V with V fragments from
+  // ldmatrix.trans.
+  const int grp = warp / kDecGroupWarps, wg = warp % kDecGroupWarps;
   const int gq = lane >> 2, cq = lane & 3;
-  int st = 0;
-  uint32_t ph = 0;
   const float NEG = -INFINITY;
+  const int nthr = kDecConsumerWarps * 32;
+  int64_t kseq = 0;  // CTA-local index of the next chunk (same order as the producer)
   for (int pr = first_pair; pr < npairs; pr += pair_step) {
     const int64_t pbeg = sm.prefix[pr], pend = sm.prefix[pr + 1];
     if (pbeg >= hi) break;
@@ -291,21 +315,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int64_t c1 = (hi < pend ? hi : pend) - pbeg;
     const bool whole = (c0 == 0) && (c1 == pend - pbeg);
 
-    // Q fragments (A operand, 16 rows x 128) for this pair
+    // Q fragments (A operand, 16 rows x 128) and per-row limits for this pair
     uint32_t qa[8][4];
+    const int r0 = gq, r1 = gq + 8;
+    const bool v0 = r0 < p.rows, v1 = r1 < p.rows;
+    // causal limit of source-A key positions for rows r0, r1
+    const int lim0 = v0 ? r0 / p.G + (p.S_A - p.Sq) : -1;
+    const int lim1 = v1 ? r1 / p.G + (p.S_A - p.Sq) : -1;
     {
-      const int r0 = gq, r1 = gq + 8;
-      const __nv_bfloat16* q0 = nullptr;
-      const __nv_bfloat16* q1 = nullptr;
-      if (r0 < p.rows) q0 = p.q + b * p.qsb + (r0 / p.G) * p.qss + (g * p.G + r0 % p.G) * p.qsh;
-      if (r1 < p.rows) q1 = p.q + b * p.qsb + (r1 / p.G) * p.qss + (g * p.G + r1 % p.G) * p.qsh;
+      const __nv_bfloat16* q0 =
+          v0 ? p.q + b * p.qsb + (r0 / p.G) * p.qss + (g * p.G + r0 % p.G) * p.qsh : nullptr;
+      const __nv_bfloat16* q1 =
+          v1 ? p.q + b * p.qsb + (r1 / p.G) * p.qss + (g * p.G + r1 % p.G) * p.qsh : nullptr;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const int d = ks * 16 + 2 * cq;
-        qa[ks][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + d) : 0u;
-        qa[ks][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + d) : 0u;
-        qa[ks][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + d + 8) : 0u;
-        qa[ks][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + d + 8) : 0u;
+        qa[ks][0] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d)) : 0u;
+        qa[ks][1] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d)) : 0u;
+        qa[ks][2] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d + 8)) : 0u;
+        qa[ks][3] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d + 8)) : 0u;
       }
     }
     float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
@@ -314,37 +342,47 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
 
     bool ok = true;
-    for (int64_t c = c0; c < c1; ++c) {
+    const int64_t k_first = kseq, k_end = kseq + (c1 - c0);
+    kseq = k_end;
+    for (int64_t kk = k_first + ((k_first & 1) != grp ? 1 : 0); kk < k_end; kk += 2) {
+      const int st = static_cast<int>(kk % kDecStages);
+      const uint32_t ph = static_cast<uint32_t>((kk / kDecStages) & 1);
       if (!mbar_wait(&sm.full[st], ph, wctx)) { ok = false; break; }
       const DecStageMeta mt = sm.meta[st];
       const uint32_t kbase = smem_u32(sm.stage[st]);
       const uint32_t vbase = kbase + kDecStageBytes / 2;
-      const int kw = warp * 16;
+      const int kw = wg * 16;
       float s[2][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-        const int key = kw + nt * 8 + gq;
+      for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      {
+        // ldmatrix x4: matrices (keys kw..+7 | kw+8..+15) x (d lo | d hi of the k-step)
+        const int mi = lane >> 3, ri = lane & 7;
+        const int key = kw + (mi >> 1) * 8 + ri;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const int d = ks * 16 + 2 * cq;
-          const uint32_t b0 = lds32(dec_elem_addr(kbase, key, d));
-          const uint32_t b1 = lds32(dec_elem_addr(kbase, key, d + 8));
-          mma_bf16_16816(s[nt], qa[ks], b0, b1);
+          uint32_t b00, b01, b10, b11;
+          const uint32_t addr = dec_elem_addr(kbase, key, ks * 16 + (mi & 1) * 8);
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(b00), "=r"(b01), "=r"(b10), "=r"(b11)
+                       : "r"(addr));
+          mma_bf16_16816(s[0], qa[ks], b00, b01);
+          mma_bf16_16816(s[1], qa[ks], b10, b11);
         }
       }
-      // scale, mask, online softmax (rows gq and gq+8)
+      // scale and mask (fast path: a full chunk that needs no causal mask)
+      const bool full_chunk = mt.nkeys >= kDecChunk &&
+                              (mt.src == 1 || !p.causal_A || mt.key0 + kDecChunk - 1 <= min(lim0, lim1 < 0 ? lim0 : lim1));
       float mx0 = NEG, mx1 = NEG;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int kk = kw + nt * 8 + 2 * cq + (e & 1);
-          const int rr = (e < 2) ? gq : gq + 8;
-          bool vis = kk < mt.nkeys && rr < p.rows;
-          if (vis && mt.src == 0 && p.causal_A) {
-            const int sqpos = rr / p.G;
-            vis = (mt.key0 + kk) <= sqpos + (p.S_A - p.Sq);
+          const int kc = kw + nt * 8 + 2 * cq + (e & 1);
+          bool vis = (e < 2) ? v0 : v1;
+          if (!full_chunk) {
+            vis = vis && kc < mt.nkeys;
+            if (mt.src == 0 && p.causal_A) vis = vis && (mt.key0 + kc) <= ((e < 2) ? lim0 : lim1);
           }
           const float x = vis ? s[nt][e] * p.scale_log2 : NEG;
           s[nt][e] = x;
@@ -355,11 +393,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float mu0 = (mn0 == NEG) ? 0.f : mn0, mu1 = (mn1 == NEG) ? 0.f : mn1;
-      const float al0 = ex2_approx(m0 - mu0), al1 = ex2_approx(m1 - mu1);
-      m0 = mn0;
-      m1 = mn1;
+      // lazy running max: raise it only when a row max exceeds it by > 2^8
+      float al0 = 1.f, al1 = 1.f;
+      if (mx0 > m0 + 8.f) { al0 = ex2_approx(m0 - mx0); m0 = mx0; }
+      if (mx1 > m1 + 8.f) { al1 = ex2_approx(m1 - mx1); m1 = mx1; }
+      const float mu0 = (m0 == NEG) ? 0.f : m0, mu1 = (m1 == NEG) ? 0.f : m1;
       float ps0 = 0.f, ps1 = 0.f;
       uint32_t pa[4];
 #pragma unroll
@@ -373,10 +411,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       l0 = l0 * al0 + ps0;
       l1 = l1 * al1 + ps1;
+      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        oacc[i][0] *= al0; oacc[i][1] *= al0;
-        oacc[i][2] *= al1; oacc[i][3] *= al1;
+        for (int i = 0; i < 16; ++i) {
+          oacc[i][0] *= al0; oacc[i][1] *= al0;
+          oacc[i][2] *= al1; oacc[i][3] *= al1;
+        }
       }
       // PV: A = P (16 x 16 keys of this warp), B = V[16 keys][128]
       {
@@ -385,47 +425,81 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int dt2 = 0; dt2 < 8; ++dt2) {
           const int d0 = dt2 * 16 + (mi >> 1) * 8;
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4_trans(dec_elem_addr(vbase, key, d0), r0, r1, r2, r3);
-          mma_bf16_16816(oacc[2 * dt2], pa, r0, r1);
-          mma_bf16_16816(oacc[2 * dt2 + 1], pa, r2, r3);
+          uint32_t x0, x1, x2, x3;
+          ldsm_x4_trans(dec_elem_addr(vbase, key, d0), x0, x1, x2, x3);
+          mma_bf16_16816(oacc[2 * dt2], pa, x0, x1);
+          mma_bf16_16816(oacc[2 * dt2 + 1], pa, x2, x3);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[st]);
-      if (++st == kDecStages) { st = 0; ph ^= 1u; }
     }
-    // ---- merge the four warps' states for this pair
-    const int nthr = kDecConsumerWarps * 32;
+    // ---- merge the eight warps' states for this pair
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (cq == 0) {
-      sm.mw[warp][gq] = m0;
-      sm.mw[warp][gq + 8] = m1;
-      sm.lw[warp][gq] = l0;
-      sm.lw[warp][gq + 8] = l1;
-    }
+    // (1) group 1 publishes its state, group 0 folds it into its registers
+    if (grp == 1) {
+      if (cq == 0) {
+        sm.mw[wg][gq] = m0; sm.mw[wg][gq + 8] = m1;
+        sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
+      }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int d = i * 8 + 2 * cq;
-      sm.ow[warp][gq][d] = oacc[i][0];
-      sm.ow[warp][gq][d + 1] = oacc[i][1];
-      sm.ow[warp][gq + 8][d] = oacc[i][2];
-      sm.ow[warp][gq + 8][d + 1] = oacc[i][3];
+      for (int i = 0; i < 16; ++i) {
+        const int d = i * 8 + 2 * cq;
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
+      }
     }
     const bool aborted = named_bar_or(1, nthr, !ok || sm.abort_flag != 0);
+    if (grp == 0 && !aborted) {
+      const float om0 = sm.mw[wg][gq], om1 = sm.mw[wg][gq + 8];
+      const float M0 = fmaxf(m0, om0), M1 = fmaxf(m1, om1);
+      const float Mu0 = (M0 == NEG) ? 0.f : M0, Mu1 = (M1 == NEG) ? 0.f : M1;
+      const float a0 = ex2_approx(m0 - Mu0), b0 = ex2_approx(om0 - Mu0);
+      const float a1 = ex2_approx(m1 - Mu1), b1 = ex2_approx(om1 - Mu1);
+      l0 = a0 * l0 + b0 * sm.lw[wg][gq];
+      l1 = a1 * l1 + b1 * sm.lw[wg][gq + 8];
+      m0 = M0;
+      m1 = M1;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int d = i * 8 + 2 * cq;
+        const float2 x = *reinterpret_cast<const float2*>(&sm.ow[wg][gq][d]);
+        const float2 y = *reinterpret_cast<const float2*>(&sm.ow[wg][gq + 8][d]);
+        oacc[i][0] = a0 * oacc[i][0] + b0 * x.x;
+        oacc[i][1] = a0 * oacc[i][1] + b0 * x.y;
+        oacc[i][2] = a1 * oacc[i][2] + b1 * y.x;
+        oacc[i][3] = a1 * oacc[i][3] + b1 * y.y;
+      }
+    }
+    named_bar_sync(1, nthr);
+    // (2) group 0 publishes the folded states
+    if (grp == 0 && !aborted) {
+      if (cq == 0) {
+        sm.mw[wg][gq] = m0; sm.mw[wg][gq + 8] = m1;
+        sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int d = i * 8 + 2 * cq;
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
+      }
+    }
+    named_bar_sync(1, nthr);
     if (!aborted) {
-      // thread t owns column d = t of every row
-      const int d = tid;
+      // 256 threads: thread t owns column d = t % 128 of rows r with r % 2 == t / 128
+      const int d = tid % kDecD;
+      const int rpar = tid / kDecD;
       const int slot = (pr == first_pair) ? 2 * cta : 2 * cta + 1;
-      for (int rr = 0; rr < p.rows; ++rr) {
+      for (int rr = rpar; rr < p.rows; rr += 2) {
         float M = NEG;
-        for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, sm.mw[w][rr]);
+        for (int w = 0; w < kDecGroupWarps; ++w) M = fmaxf(M, sm.mw[w][rr]);
         const float Mu = (M == NEG) ? 0.f : M;
         float L = 0.f, acc = 0.f;
-        for (int w = 0; w < kDecConsumerWarps; ++w) {
+        for (int w = 0; w < kDecGroupWarps; ++w) {
           const float wt = ex2_approx(sm.mw[w][rr] - Mu);
           L += wt * sm.lw[w][rr];
           acc += wt * sm.ow[w][rr][d];
@@ -455,7 +529,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (sm.is_last) {
           const int c_first = dec_cta_of(pbeg, total, grid);
           const int c_last = dec_cta_of(pend - 1, total, grid);
-          for (int rr = 0; rr < p.rows; ++rr) {
+          for (int rr = rpar; rr < p.rows; rr += 2) {
             float M = NEG;
             for (int cc = c_first; cc <= c_last; ++cc) {
               if (dec_range_lo(cc, total, grid) == dec_range_lo(cc + 1, total, grid)) continue;

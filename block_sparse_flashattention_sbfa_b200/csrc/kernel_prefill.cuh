@@ -78,6 +78,7 @@ struct PrefillParams {
   const __nv_bfloat16* v;
   int64_t ksb, kss, ksh, vsb, vss, vsh;
   int* status;
+  unsigned long long* prof;  // 32 counters, self-profiling build only
 };
 
 struct PfSched {
@@ -113,7 +114,7 @@ struct PfSmem {
 // Visit the union of the four segments' tile sets in ascending order, then the
 // vertical-column chunks.  fn(item, kt_or_chunk, is_col, mem) with mem = bit s
 // set when segment s takes part; stops early when fn returns false.
-template <class F>
+template <bool COLS, class F>
 __device__ __forceinline__ bool pf_for_each(const PfSched& sc, F&& fn) {
   int item = 0;
   for (int w = 0; w < sc.n_words; ++w) {
@@ -127,6 +128,7 @@ __device__ __forceinline__ bool pf_for_each(const PfSched& sc, F&& fn) {
       if (!fn(item++, w * 32 + bit, false, mem)) return false;
     }
   }
+  if (!COLS) return true;
   const int nch = (sc.n_cols + 63) >> 6;
   for (int c = 0; c < nch; ++c) {
     int mem = 0;
@@ -267,6 +269,7 @@ __device__ __forceinline__ void pf_gather_rows(const PfSched& sc, int c, const _
   __syncwarp();
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
                    const __grid_constant__ CUtensorMap mapK,
@@ -316,7 +319,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wctx{&sm.abort_flag, p.status};
-  const bool gated = p.mode == kModeGated;
+  constexpr bool gated = MODE == kModeGated;
+  constexpr bool has_cols = MODE == kModeVS;
+  unsigned long long pacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const long long t_start = clock64();
 
   if (warp == 0) {
     // ============================ Q/K producer ============================
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       pf_build_sched(p, u, sc, lane);
       if (lane == 0) {
         mbar_arrive(&sm.sched_full[ub]);
-        ok = mbar_wait(&sm.q_empty, (n & 1) ^ 1u, wctx);
+        ok = mbar_wait_t(&sm.q_empty, (n & 1) ^ 1u, wctx, pacc[1]);
         if (ok) {
           for (int t = 0; t < 2; ++t) {
             const int nv = sc.seg_valid[2 * t] + sc.seg_valid[2 * t + 1];
@@ -357,10 +363,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!ok) break;
       auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
         bool good = true;
-        if (lane == 0) good = mbar_wait(&sm.k_empty[ks], kph ^ 1u, wctx);
+        if (lane == 0) good = mbar_wait_t(&sm.k_empty[ks], kph ^ 1u, wctx, pacc[0]);
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
         if (!good) return false;
-        if (!is_col) {
+        if (!has_cols || !is_col) {
           if (lane == 0) {
             mbar_arrive_expect_tx(&sm.k_full[ks], kTileBytes);
             tma_load_4d(sm.k[ks], &mapK, &sm.k_full[ks], 0, sc.g, kt * 64, sc.b);
@@ -373,7 +379,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (++ks == kKStages) { ks = 0; kph ^= 1u; }
         return true;
       };
-      ok = pf_for_each(sc, body);
+      ok = pf_for_each<has_cols>(sc, body);
     }
     if (!ok && lane == 0)
       for (int i = 0; i < kKStages; ++i) mbar_wait_short(&sm.k_full[i], 0);
@@ -396,7 +402,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int need = 1;
         if (gated) {
           if (lane == 0) {
-            good = mbar_wait(&sm.dec_full[dslot], dph, wctx);
+            good = mbar_wait_t(&sm.dec_full[dslot], dph, wctx, pacc[1]);
             if (good) {
               need = sm.dec_val[dslot][0] | sm.dec_val[dslot][1];
               mbar_arrive(&sm.dec_empty[dslot]);
@@ -408,10 +414,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (!good) return false;
           if (!need) return true;
         }
-        if (lane == 0) good = mbar_wait(&sm.v_empty[vs], vph ^ 1u, wctx);
+        if (lane == 0) good = mbar_wait_t(&sm.v_empty[vs], vph ^ 1u, wctx, pacc[0]);
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
         if (!good) return false;
-        if (!is_col) {
+        if (!has_cols || !is_col) {
           if (lane == 0) {
             mbar_arrive_expect_tx(&sm.v_full[vs], kTileBytes);
             tma_load_4d(sm.v[vs], &mapV, &sm.v_full[vs], 0, sc.g, kt * 64, sc.b);
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (++vs == kVStages) { vs = 0; vph ^= 1u; }
         return true;
       };
-      ok = pf_for_each(sc, body);
+      ok = pf_for_each<has_cols>(sc, body);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sched_empty[ub]);
     }
@@ -449,7 +455,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         PfSched& sc = sm.sched[ub];
         ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
         if (!ok) break;
-        ok = mbar_wait(&sm.q_full[0], n & 1, wctx) && mbar_wait(&sm.q_full[1], n & 1, wctx);
+        ok = mbar_wait_t(&sm.q_full[0], n & 1, wctx, pacc[5]) &&
+             mbar_wait_t(&sm.q_full[1], n & 1, wctx, pacc[5]);
         if (!ok) break;
         int pv_started[2] = {0, 0};
         int ofree_waited[2] = {0, 0};
@@ -459,18 +466,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int t = 0; t < 2; ++t) {
             if (!((act >> t) & 1)) continue;
             const int sl = pslot[t];
-            if (!mbar_wait(&sm.p_full[t][sl], pph[t][sl], wctx)) return false;
+            if (!mbar_wait_t(&sm.p_full[t][sl], pph[t][sl], wctx, pacc[2])) return false;
             pph[t][sl] ^= 1u;
             flag[t] = sm.pv_flag[t][sl];
             pslot[t] ^= 1;
           }
           if (!(flag[0] | flag[1])) return true;
-          if (!mbar_wait(&sm.v_full[vs], vph, wctx)) return false;
+          if (!mbar_wait_t(&sm.v_full[vs], vph, wctx, pacc[3])) return false;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
             if (!flag[t]) continue;
             if (!ofree_waited[t]) {
-              if (!mbar_wait(&sm.o_free[t], ofph[t] ^ 1u, wctx)) return false;
+              if (!mbar_wait_t(&sm.o_free[t], ofph[t] ^ 1u, wctx, pacc[4])) return false;
               ofph[t] ^= 1u;
               ofree_waited[t] = 1;
               tc_fence_after();
@@ -493,12 +500,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
           const int act = ((mem & 3) ? 1 : 0) | ((mem & 12) ? 2 : 0);
-          if (!mbar_wait(&sm.k_full[ks], kph, wctx)) return false;
+          if (!mbar_wait_t(&sm.k_full[ks], kph, wctx, pacc[0])) return false;
+          pacc[7] += 1;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
             if (!((act >> t) & 1)) continue;
             const int bsel = sbuf[t];
-            if (!mbar_wait(&sm.s_empty[t][bsel], sph[t][bsel] ^ 1u, wctx)) return false;
+            if (!mbar_wait_t(&sm.s_empty[t][bsel], sph[t][bsel] ^ 1u, wctx, pacc[1])) return false;
             sph[t][bsel] ^= 1u;
             tc_fence_after();
             const uint32_t d_tmem = tmem + t * 256 + bsel * 64;
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           prev_act = act;
           return true;
         };
-        ok = pf_for_each(sc, body);
+        ok = pf_for_each<has_cols>(sc, body);
         if (ok && prev_act) ok = do_pv(prev_act);
         for (int t = 0; t < 2 && ok; ++t) {
           if (!ofree_waited[t]) {
@@ -568,7 +576,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!tile_act) {
           if (gated) {
             if (tid == 128 + 128 * t) {
-              if (!mbar_wait(&sm.dec_empty[dslot], dph ^ 1u, wctx)) return false;
+              if (!mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2])) return false;
               sm.dec_val[dslot][t] = 0;
               mbar_arrive(&sm.dec_full[dslot]);
             }
@@ -577,40 +585,41 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           return true;
         }
         const bool seg_act = ((mem >> seg) & 1) && my_row < p.Sq;
-        if (!mbar_wait(&sm.s_full[t][sbuf], (sphase >> sbuf) & 1u, wctx)) return false;
+        if (!mbar_wait_t(&sm.s_full[t][sbuf], (sphase >> sbuf) & 1u, wctx, pacc[0])) return false;
         sphase ^= 1u << sbuf;
         tc_fence_after();
         float s[64];
-        tmem_ld32(lane_addr + sbuf * 64, s);
-        tmem_ld32(lane_addr + sbuf * 64 + 32, s + 32);
+        tmem_ld64(lane_addr + sbuf * 64, s);
         tc_fence_before();
         mbar_arrive(&sm.s_empty[t][sbuf]);
         sbuf ^= 1;
-        // ---- masks
+        pacc[5] += 1;
+        // ---- masks: row max over the visible keys of this tile
         float rmax = NEG;
-        if (!is_col) {
-          const int key0 = kt * 64;
-          const bool need =
-              (p.causal && key0 + 63 > my_row + p.causal_off) || (key0 + 64 > p.Sk);
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            bool vis = seg_act;
-            if (need) {
-              const int key = key0 + c;
-              vis = vis && key < p.Sk && (!p.causal || key <= my_row + p.causal_off);
-            }
-            s[c] = vis ? s[c] : NEG;
-            rmax = fmaxf(rmax, s[c]);
-          }
-        } else {
+        if (has_cols && is_col) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             const int e = kt * 64 + c;
             bool vis = seg_act && e < sc.n_cols && ((sc.colmask[e] >> seg) & 1);
             if (vis && p.causal) vis = sc.col[e] <= my_row + p.causal_off;
             s[c] = vis ? s[c] : NEG;
-            rmax = fmaxf(rmax, s[c]);
           }
+        } else {
+          // keys [key0, key0 + lim) of this tile are visible to the row
+          const int key0 = kt * 64;
+          int lim = seg_act ? 64 : 0;
+          lim = min(lim, p.Sk - key0);
+          if (p.causal) lim = min(lim, my_row + p.causal_off - key0 + 1);
+          if (lim < 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = (c < lim) ? s[c] : NEG;
+          }
+        }
+        {
+          float m4[4] = {NEG, NEG, NEG, NEG};
+#pragma unroll
+          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+          rmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         bool my_keep = seg_act;
         bool tile_keep = true;
@@ -644,7 +653,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           my_keep = hseg ? keep2[1] : keep2[0];
           tile_keep = keep2[0] || keep2[1];
           if (r == 0) {
-            if (!mbar_wait(&sm.dec_empty[dslot], dph ^ 1u, wctx)) return false;
+            if (!mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2])) return false;
             sm.dec_val[dslot][t] = tile_keep ? 1 : 0;
             mbar_arrive(&sm.dec_full[dslot]);
           }
@@ -668,23 +677,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
         const float mu = (m_used == NEG) ? 0.f : m_used;
-        float psum = 0.f;
         uint32_t pk[32];
+        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (my_keep) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (my_keep) {
-            p0 = ex2_approx(fmaf(s[c], p.scale_log2, -mu));
-            p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -mu));
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -mu));
+            const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -mu));
+            ps4[(c >> 1) & 3] += p0 + p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
           }
-          psum += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
-        l = l * alpha + psum;
+        l = l * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
         if (npv > 0) {
-          if (!mbar_wait(&sm.pv_done[t], (pv_total - 1) & 1, wctx)) return false;
+          if (!mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1])) return false;
           tc_fence_after();
           if (__any_sync(0xffffffffu, resc)) {
+            pacc[6] += 1;
             float ob[32];
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
@@ -711,9 +723,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         pslot ^= 1;
         ++npv;
         ++pv_total;
+        pacc[7] += 1;
         return true;
       };
-      ok = pf_for_each(sc, body);
+      ok = pf_for_each<has_cols>(sc, body);
       if (!ok) break;
       // ---- epilogue: o = O / l, lse = ln(sum)
       const bool store = my_valid && my_row < p.Sq;
@@ -763,6 +776,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   }
   // warp 3 idles (reserved)
+#if SBFA_PROF_ON
+  if (p.prof) {
+    int base = -1;
+    if (tid == 0) base = 0;            // Q/K producer
+    else if (tid == 64) base = 8;      // V producer
+    else if (tid == 32) base = 16;     // MMA issuer
+    else if (tid == 128) base = 24;    // softmax tile 0
+    if (base >= 0) {
+      for (int i = 0; i < 7; ++i) atomicAdd(p.prof + base + i, pacc[i]);
+      atomicAdd(p.prof + base + 7, pacc[7]);
+      if (base == 24) atomicAdd(p.prof + 32, static_cast<unsigned long long>(clock64() - t_start));
+    }
+  }
+#else
+  (void)t_start;
+#endif
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

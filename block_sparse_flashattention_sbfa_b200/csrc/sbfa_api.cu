@@ -141,6 +141,10 @@ float eff_scale(const sbfa_shape* s) {
     if (st_ != SBFA_OK) return st_; \
   } while (0)
 
+// Device counters of the self-profiling build (null otherwise); set through
+// sbfa_set_profile_counters, which only that build exports.
+unsigned long long* g_prof_counters = nullptr;
+
 // ---------------------------------------------------------------------------
 // prefill launcher (tcgen05 kernel)
 // ---------------------------------------------------------------------------
@@ -176,16 +180,37 @@ sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sb
   SBFA_TRY(encode_bshd(&mk, k, s->B, s->Sk, s->Hkv, 64));
   SBFA_TRY(encode_bshd(&mv, v, s->B, s->Sk, s->Hkv, 64));
   const size_t smem = sizeof(sbfa::PfSmem) + 1024;
-  static bool attr_set[64] = {false};
+  static bool attr_set[64][4] = {};
   int dev = 0;
   SBFA_CUDA(cudaGetDevice(&dev));
-  if (!attr_set[dev]) {
-    SBFA_CUDA(cudaFuncSetAttribute(sbfa::prefill_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr_set[dev] = true;
+  const void* fn = nullptr;
+  switch (p.mode) {
+    case sbfa::kModeTable: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeTable>); break;
+    case sbfa::kModeDense: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeDense>); break;
+    case sbfa::kModeGated: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeGated>); break;
+    case sbfa::kModeVS: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeVS>); break;
+    default: return fail(SBFA_ERR_INVALID_ARG, "internal: bad prefill mode");
   }
+  if (!attr_set[dev][p.mode]) {
+    SBFA_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr_set[dev][p.mode] = true;
+  }
+  p.prof = g_prof_counters;
   const int grid = std::min(p.n_units, di.sms);
-  sbfa::prefill_kernel<<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
+  switch (p.mode) {
+    case sbfa::kModeTable:
+      sbfa::prefill_kernel<sbfa::kModeTable><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
+      break;
+    case sbfa::kModeDense:
+      sbfa::prefill_kernel<sbfa::kModeDense><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
+      break;
+    case sbfa::kModeGated:
+      sbfa::prefill_kernel<sbfa::kModeGated><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
+      break;
+    default:
+      sbfa::prefill_kernel<sbfa::kModeVS><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
+      break;
+  }
   SBFA_CUDA(cudaGetLastError());
   return SBFA_OK;
 }
@@ -383,6 +408,12 @@ extern "C" {
 const char* sbfa_last_error(void) { return g_last_error.c_str(); }
 
 const char* sbfa_version(void) { return "sbfa 0.1 (sm_100a)"; }
+
+#ifdef SBFA_PROFILE
+// Self-profiling build only: device array of 33 uint64 counters that the
+// prefill kernel adds its per-role wait cycles to (null disables).
+void sbfa_set_profile_counters(unsigned long long* counters) { g_prof_counters = counters; }
+#endif
 
 sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
                      const sbfa_table* table, sbfa_t4 o, float* lse, int32_t* status,
