@@ -251,6 +251,10 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
+      const uint64_t qdesc0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.v[0]), 8192, 1024);
+      const uint64_t pdesc0 = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
       bool ok = true;
       auto issue_qk = [&](int n) -> bool {
         const int b = n & 1;
@@ -258,12 +262,13 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         if (!mbar_wait(&sm.q_full[b], ph, wctx) || !mbar_wait(&sm.kv_full[b], ph, wctx))
           return false;
         tc_fence_after();
-        const uint32_t qa = smem_u32(sm.q[b]), ka = smem_u32(sm.k[b]);
+        const uint64_t qd = qdesc0 + (b * kQTileBytes >> 4);
+        const uint64_t kd = kdesc0 + (b * kTileBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          umma_ss(tmem + b * 256, ad, bd, idesc_qk, kk ? 1u : 0u);
+          const uint32_t off_q = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          const uint32_t off_k = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + b * 256, qd + off_q, kd + off_k, idesc_qk, kk ? 1u : 0u);
         }
         umma_commit(&sm.s_full[b]);
         return true;
@@ -273,13 +278,12 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         const uint32_t ph = (n >> 1) & 1;
         if (!mbar_wait(&sm.p_full[b], ph, wctx)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sm.p[b]), va = smem_u32(sm.v[b]);
+        const uint64_t pd = pdesc0 + (b * kPTileBytes >> 4);
+        const uint64_t vd = vdesc0 + (b * kTileBytes >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = sdesc_sw128(pa + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(va + kk * 2048, 8192, 1024);
-          umma_ss(tmem + b * 256 + 128, ad, bd, idesc_pv, kk ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ss(tmem + b * 256 + 128, pd + (kk * 32 >> 4), vd + (kk * 2048 >> 4), idesc_pv,
+                  kk ? 1u : 0u);
         umma_commit(&sm.o_full[b]);
         return true;
       };
@@ -319,7 +323,8 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         tl = t - base;
         L = __ldg(p.cu + un.s + 1) - base;
       }
-      if (!mbar_wait(&sm.s_full[b], ph, wctx)) { ok = false; break; }
+      // tcgen05.ld is warp-collective: the warp agrees before leaving
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], ph, wctx))) { ok = false; break; }
       tc_fence_after();
       float s[64];
       tmem_ld32(lane_addr, s);
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.p_full[b]);
-      if (!mbar_wait(&sm.o_full[b], ph, wctx)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[b], ph, wctx))) { ok = false; break; }
       tc_fence_after();
       const int h = un.g * p.G + r % p.G;
       const int64_t prow_idx = (static_cast<int64_t>(t) * p.Hq + h) * p.topk + slot;

@@ -1,13 +1,14 @@
 // Block-sparse FlashAttention forward on the 5th-generation tensor cores.
 //
-// One persistent CTA per SM, warp-specialised:
+// One persistent CTA per SM, warp-specialised (384 threads):
 //   warp 0      TMA producer for Q and K tiles; builds each work unit's
-//               key-tile schedule in shared memory
-//   warp 1      tcgen05 MMA issuer (one elected lane); owns the TMEM allocation
-//   warp 2      producer for V tiles (waits for the gate's keep decision in
-//               gated mode: pruned blocks load no V, BSFA Figure 2b) and for
-//               gathered vertical columns
-//   warp 3      gathers K rows of vertical columns
+//               key-tile schedule in shared memory; gathers K rows of
+//               vertical columns
+//   warp 1      tcgen05 MMA issuer (one lane); owns the TMEM allocation
+//   warp 2      producer for V tiles -- in gated mode it waits for the
+//               gate's keep decision and loads no V for pruned blocks (BSFA
+//               Figure 2b); gathers V rows of vertical columns
+//   warp 3      idle
 //   warps 4-7   softmax warpgroup of Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup of Q tile 1
 //
@@ -15,18 +16,23 @@
 // with GQA they are heads of one group at the same q-block (K/V tiles are
 // loaded once for all of them); without GQA they are four consecutive
 // q-blocks of one head.  Segments 0,1 form M = 128 tile 0 and segments 2,3
-// tile 1.  Each segment has a set of 64-key tiles (from the block table, the
+// tile 1.  Each segment has a set of 64-key blocks (from the block table, the
 // causal range, the gate candidates or the vertical/slash lists); the unit
-// walks the union of the four sets in ascending order and runs
-//   S_t = Q_t K^T  (tcgen05.mma, M128 N64 K128, fp32 in TMEM)
-//   softmax rows, P_t (bf16) -> shared memory
-//   O_t += P_t V   (tcgen05.mma, M128 N128 K64, fp32 in TMEM)
-// for every tile t with an active segment; rows of an inactive segment get
-// P = 0.  The online softmax keeps a lazily updated running max (rescale O
-// only when the max grows by more than 2^8), which leaves o and lse exact.
+// walks the 128-key tiles that hold a block of any segment, in ascending
+// order, and for each tile t with an active segment runs
+//   S_t = Q_t K^T        tcgen05.mma M128 N128 K16 x 8, fp32 in TMEM
+//   softmax rows; P_t (bf16) written back over S_t in TMEM
+//   O_t += P_t V         tcgen05.mma with A from TMEM, M128 N128 K16 x 8
+// The two 64-key halves of a tile are tracked separately: a half that no
+// segment of a tile keeps contributes no PV instructions, and a half that no
+// segment of the unit keeps loads no V.  Rows of an inactive segment or half
+// get P = 0.  The online softmax keeps a lazily raised running max (O is
+// rescaled only when a row max grows by more than 2^8), which leaves o and
+// lse exact.  MMAs of one thread execute in issue order, so the commit that
+// signals S_t(e) also proves that PV_t(e-1) has read P_t(e-1) and written O_t.
 //
-// TMEM (512 columns): tile t uses columns [256t, 256t+256): S buffers 0/1 at
-// +0/+64 (64 fp32 columns each), O at +128 (128 columns).
+// TMEM (512 columns): tile t uses [256t, 256t+128) for S (fp32) / P (bf16
+// pairs, first 64 columns) and [256t+128, 256t+256) for O.
 #pragma once
 
 #include "sbfa_ptx.cuh"
@@ -36,13 +42,14 @@ namespace sbfa {
 enum PrefillMode : int { kModeTable = 0, kModeDense = 1, kModeGated = 2, kModeVS = 3 };
 
 constexpr int kPfThreads = 384;
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
-constexpr int kMaxKT = 8192;              // 64-key tiles: Sk <= 524288
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
+constexpr int kMaxKT = 8192;               // 64-key blocks: Sk <= 524288
 constexpr int kBmWords = kMaxKT / 32;
 constexpr int kDecRingSlots = 4;
-constexpr int kMaxCols = 1024;            // union of vertical columns per unit
-constexpr int kTileBytes = 64 * 128 * 2;  // 64 keys x 128 dims bf16
+constexpr int kMaxCols = 1024;             // union of vertical columns per unit
+constexpr int kTileBytes = 64 * 128 * 2;   // 64 keys x 128 dims bf16
+constexpr int kKVTileBytes = 128 * 128 * 2;  // 128 keys: [d-chunk][128 rows][128 B]
 constexpr int kQTileBytes = 128 * 128 * 2;
 constexpr int kPTileBytes = 128 * 64 * 2;
 
@@ -93,48 +100,59 @@ struct PfSched {
 
 struct PfSmem {
   alignas(1024) uint8_t q[2][kQTileBytes];
-  alignas(1024) uint8_t k[kKStages][kTileBytes];
-  alignas(1024) uint8_t v[kVStages][kTileBytes];
-  alignas(1024) uint8_t p[2][kPTileBytes];
+  alignas(1024) uint8_t k[kKStages][kKVTileBytes];
+  alignas(1024) uint8_t v[kVStages][kKVTileBytes];
   PfSched sched[2];
-  float red[2][2][4];
+  float red[2][2][4][2];      // [tile][parity][warp][half] block-max exchange
   int dec_val[kDecRingSlots][2];
-  int pv_flag[2][2];
+  int pv_flag[2];
   uint32_t tmem_base;
   int abort_flag;
   uint64_t sched_full[2], sched_empty[2];
   uint64_t q_full[2], q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2][2], s_empty[2][2];
-  uint64_t p_full[2][2], pv_done[2], o_free[2];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
   uint64_t dec_full[kDecRingSlots], dec_empty[kDecRingSlots];
 };
 
-// Visit the union of the four segments' tile sets in ascending order, then the
-// vertical-column chunks.  fn(item, kt_or_chunk, is_col, mem) with mem = bit s
-// set when segment s takes part; stops early when fn returns false.
+static_assert(sizeof(PfSmem) + 1024 <= 232448, "prefill shared memory exceeds 227 KB");
+
+// Visit the 128-key tiles that hold a 64-key block of any segment (ascending),
+// then the vertical-column chunks of 128.  fn(kt, is_col, mem) where bit
+// (2s + h) of mem says segment s takes part in half h; stops when fn
+// returns false.
 template <bool COLS, class F>
 __device__ __forceinline__ bool pf_for_each(const PfSched& sc, F&& fn) {
-  int item = 0;
   for (int w = 0; w < sc.n_words; ++w) {
-    const uint32_t b0 = sc.bm[0][w], b1 = sc.bm[1][w], b2 = sc.bm[2][w], b3 = sc.bm[3][w];
-    uint32_t any = b0 | b1 | b2 | b3;
+    uint32_t bits[4];
+    uint32_t any = 0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      bits[s] = sc.bm[s][w];
+      any |= (bits[s] | (bits[s] >> 1)) & 0x55555555u;
+    }
     while (any) {
-      const int bit = __ffs(any) - 1;
+      const int bit = __ffs(any) - 1;  // even: half 0 of tile (32w + bit) / 2
       any &= any - 1u;
-      const int mem = ((b0 >> bit) & 1) | (((b1 >> bit) & 1) << 1) | (((b2 >> bit) & 1) << 2) |
-                      (((b3 >> bit) & 1) << 3);
-      if (!fn(item++, w * 32 + bit, false, mem)) return false;
+      int mem = 0;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mem |= ((bits[s] >> bit) & 3) << (2 * s);
+      if (!fn((w * 32 + bit) >> 1, false, mem)) return false;
     }
   }
   if (!COLS) return true;
-  const int nch = (sc.n_cols + 63) >> 6;
+  const int nch = (sc.n_cols + 127) >> 7;
   for (int c = 0; c < nch; ++c) {
     int mem = 0;
-    const int e1 = min(sc.n_cols, c * 64 + 64);
-    for (int e = c * 64; e < e1; ++e) mem |= sc.colmask[e];
-    if (!fn(item++, c, true, mem)) return false;
+    for (int h = 0; h < 2; ++h) {
+      const int e0 = c * 128 + h * 64, e1 = min(sc.n_cols, e0 + 64);
+      int m = 0;
+      for (int e = e0; e < e1; ++e) m |= sc.colmask[e];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mem |= ((m >> s) & 1) << (2 * s + h);
+    }
+    if (!fn(c, true, mem)) return false;
   }
   return true;
 }
@@ -244,18 +262,17 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
   __syncwarp();
 }
 
-// Gather 64 K or V rows (vertical columns of chunk c) into a swizzled tile;
-// rows past the list end are zero-filled.  Whole warp; completes the
-// copies and the proxy fence before returning.
-__device__ __forceinline__ void pf_gather_rows(const PfSched& sc, int c, const __nv_bfloat16* base,
-                                               int64_t sb, int64_t ss, int64_t sh, uint8_t* dst,
-                                               int lane) {
-  const uint32_t d0 = smem_u32(dst);
+// Gather 64 K or V rows (vertical columns e0 .. e0+63 of the union list)
+// into half `half` of a 128-key tile; rows past the list end are zero.
+// Whole warp; completes the copies and the proxy fence before returning.
+__device__ __forceinline__ void pf_gather_rows(const PfSched& sc, int e0, int half,
+                                               const __nv_bfloat16* base, int64_t sb, int64_t ss,
+                                               int64_t sh, uint8_t* dst, int lane) {
+  const uint32_t d0 = smem_u32(dst) + half * 8192;
   for (int e = lane; e < 64 * 16; e += 32) {
     const int r = e >> 4, ch = e & 15;  // row, 16-byte chunk of the 256-byte row
-    const int half = ch >> 3, cc = ch & 7;
-    const uint32_t saddr = d0 + half * 8192 + sw128_off(r, cc);
-    const int idx = c * 64 + r;
+    const uint32_t saddr = d0 + (ch >> 3) * 16384 + sw128_off(r, ch & 7);
+    const int idx = e0 + r;
     if (idx < sc.n_cols) {
       const __nv_bfloat16* src = base + sc.b * sb + static_cast<int64_t>(sc.col[idx]) * ss +
                                  sc.g * sh + ch * 8;
@@ -269,6 +286,12 @@ __device__ __forceinline__ void pf_gather_rows(const PfSched& sc, int c, const _
   __syncwarp();
 }
 
+// Halves of a 128-key tile that tile t (segments 2t, 2t+1) takes part in.
+__device__ __forceinline__ int pf_tile_halves(int mem, int t) {
+  const int m = (mem >> (4 * t)) & 15;
+  return (m | (m >> 2)) & 3;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
@@ -279,20 +302,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  constexpr bool gated = MODE == kModeGated;
+  constexpr bool has_cols = MODE == kModeVS;
+  unsigned long long pacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const long long t_start = clock64();
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sched_full[i], 1);
       mbar_init(&sm.sched_empty[i], 1 + 1 + 256);
       mbar_init(&sm.q_full[i], 1);
-      mbar_init(&sm.p_full[i][0], 128);
-      mbar_init(&sm.p_full[i][1], 128);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 128);
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.o_free[i], 128);
-      for (int j = 0; j < 2; ++j) {
-        mbar_init(&sm.s_full[i][j], 1);
-        mbar_init(&sm.s_empty[i][j], 128);
-      }
     }
     mbar_init(&sm.q_empty, 1);
     for (int i = 0; i < kKStages; ++i) {
@@ -310,6 +333,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     sm.abort_flag = 0;
     fence_mbar_init();
   }
+  // V stages start finite (zero); afterwards they only ever hold loaded rows
+  for (int i = tid; i < kVStages * kKVTileBytes / 16; i += kPfThreads)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(smem_u32(sm.v[0]) + 16 * i),
+                 "r"(0)
+                 : "memory");
+  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
@@ -319,10 +348,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wctx{&sm.abort_flag, p.status};
-  constexpr bool gated = MODE == kModeGated;
-  constexpr bool has_cols = MODE == kModeVS;
-  unsigned long long pacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  const long long t_start = clock64();
 
   if (warp == 0) {
     // ============================ Q/K producer ============================
@@ -361,19 +386,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
+      auto body = [&](int kt, bool is_col, int mem) -> bool {
         bool good = true;
         if (lane == 0) good = mbar_wait_t(&sm.k_empty[ks], kph ^ 1u, wctx, pacc[0]);
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
         if (!good) return false;
+        const int halves = (mem | (mem >> 2) | (mem >> 4) | (mem >> 6)) & 3;
         if (!has_cols || !is_col) {
           if (lane == 0) {
-            mbar_arrive_expect_tx(&sm.k_full[ks], kTileBytes);
-            tma_load_4d(sm.k[ks], &mapK, &sm.k_full[ks], 0, sc.g, kt * 64, sc.b);
-            tma_load_4d(sm.k[ks] + 8192, &mapK, &sm.k_full[ks], 64, sc.g, kt * 64, sc.b);
+            mbar_arrive_expect_tx(&sm.k_full[ks], __popc(halves) * 2 * 8192);
+            for (int h = 0; h < 2; ++h) {
+              if (!((halves >> h) & 1)) continue;
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d(sm.k[ks] + c * 16384 + h * 8192, &mapK, &sm.k_full[ks], c * 64, sc.g,
+                            kt * 128 + h * 64, sc.b);
+            }
           }
         } else {
-          pf_gather_rows(sc, kt, p.k, p.ksb, p.kss, p.ksh, sm.k[ks], lane);
+          for (int h = 0; h < 2; ++h)
+            if ((halves >> h) & 1)
+              pf_gather_rows(sc, kt * 128 + h * 64, h, p.k, p.ksb, p.kss, p.ksh, sm.k[ks], lane);
           if (lane == 0) mbar_arrive(&sm.k_full[ks]);
         }
         if (++ks == kKStages) { ks = 0; kph ^= 1u; }
@@ -397,9 +429,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (lane == 0) ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
+      auto body = [&](int kt, bool is_col, int mem) -> bool {
         bool good = true;
-        int need = 1;
+        int need = (mem | (mem >> 2) | (mem >> 4) | (mem >> 6)) & 3;
         if (gated) {
           if (lane == 0) {
             good = mbar_wait_t(&sm.dec_full[dslot], dph, wctx, pacc[1]);
@@ -412,19 +444,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
           need = __shfl_sync(0xffffffffu, need, 0);
           if (!good) return false;
-          if (!need) return true;
         }
+        if (!need) return true;
         if (lane == 0) good = mbar_wait_t(&sm.v_empty[vs], vph ^ 1u, wctx, pacc[0]);
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
         if (!good) return false;
         if (!has_cols || !is_col) {
           if (lane == 0) {
-            mbar_arrive_expect_tx(&sm.v_full[vs], kTileBytes);
-            tma_load_4d(sm.v[vs], &mapV, &sm.v_full[vs], 0, sc.g, kt * 64, sc.b);
-            tma_load_4d(sm.v[vs] + 8192, &mapV, &sm.v_full[vs], 64, sc.g, kt * 64, sc.b);
+            mbar_arrive_expect_tx(&sm.v_full[vs], __popc(need) * 2 * 8192);
+            for (int h = 0; h < 2; ++h) {
+              if (!((need >> h) & 1)) continue;
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d(sm.v[vs] + c * 16384 + h * 8192, &mapV, &sm.v_full[vs], c * 64, sc.g,
+                            kt * 128 + h * 64, sc.b);
+            }
           }
         } else {
-          pf_gather_rows(sc, kt, p.v, p.vsb, p.vss, p.vsh, sm.v[vs], lane);
+          for (int h = 0; h < 2; ++h)
+            if ((need >> h) & 1)
+              pf_gather_rows(sc, kt * 128 + h * 64, h, p.v, p.vsb, p.vss, p.vsh, sm.v[vs], lane);
           if (lane == 0) mbar_arrive(&sm.v_full[vs]);
         }
         if (++vs == kVStages) { vs = 0; vph ^= 1u; }
@@ -439,15 +477,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp == 1) {
     // ============================= MMA issuer =============================
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16(128, 64, 0);
+      const uint32_t idesc_qk = idesc_bf16(128, 128, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
+      // base descriptors; K-step and stage offsets are added to the start
+      // address field (bits 0-13, 16-byte units), which cannot overflow inside
+      // the shared window
+      const uint64_t qdesc0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.v[0]), 16384, 1024);
       int ks = 0, vs = 0;
       uint32_t kph = 0, vph = 0;
-      int sbuf[2] = {0, 0};
-      uint32_t sph[2][2] = {{0, 0}, {0, 0}};
-      uint32_t pph[2][2] = {{0, 0}, {0, 0}};
-      int pslot[2] = {0, 0};
-      uint32_t ofph[2] = {0, 0};
+      uint32_t pph = 0;   // bit t: p_full[t] phase
+      uint32_t ofph = 0;  // bit t: o_free[t] phase
       bool ok = true;
       int n = 0;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
@@ -458,87 +499,103 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ok = mbar_wait_t(&sm.q_full[0], n & 1, wctx, pacc[5]) &&
              mbar_wait_t(&sm.q_full[1], n & 1, wctx, pacc[5]);
         if (!ok) break;
-        int pv_started[2] = {0, 0};
-        int ofree_waited[2] = {0, 0};
-        int prev_act = 0;  // bit t: tile t took part in the previous item
-        auto do_pv = [&](int act) -> bool {
-          int flag[2] = {0, 0};
-          for (int t = 0; t < 2; ++t) {
-            if (!((act >> t) & 1)) continue;
-            const int sl = pslot[t];
-            if (!mbar_wait_t(&sm.p_full[t][sl], pph[t][sl], wctx, pacc[2])) return false;
-            pph[t][sl] ^= 1u;
-            flag[t] = sm.pv_flag[t][sl];
-            pslot[t] ^= 1;
+        int pv_started = 0;    // bit t
+        int ofree_waited = 0;  // bit t
+        // Issue order (two-tile ping-pong): QK(e,t0), PV(e-1,t1), QK(e,t1),
+        // PV(e,t0).  Each softmax warpgroup then computes while the tensor core
+        // runs the other tile's work.  The V stage of item e is released after
+        // PV(e,t1), which is issued while handling item e+1.
+        struct Pending {
+          int valid, act1, f0, v_waited;
+        } pend = {0, 0, 0, 0};
+        auto issue_pv = [&](int t, int flag) -> bool {
+          if (!((ofree_waited >> t) & 1)) {
+            if (!mbar_wait_t(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx, pacc[4])) return false;
+            ofph ^= 1u << t;
+            ofree_waited |= 1 << t;
+            tc_fence_after();
           }
-          if (!(flag[0] | flag[1])) return true;
-          if (!mbar_wait_t(&sm.v_full[vs], vph, wctx, pacc[3])) return false;
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (!flag[t]) continue;
-            if (!ofree_waited[t]) {
-              if (!mbar_wait_t(&sm.o_free[t], ofph[t] ^ 1u, wctx, pacc[4])) return false;
-              ofph[t] ^= 1u;
-              ofree_waited[t] = 1;
-              tc_fence_after();
-            }
-            const uint32_t d_tmem = tmem + t * 256 + 128;
-            const uint32_t pa = smem_u32(sm.p[t]);
-            const uint32_t va = smem_u32(sm.v[vs]);
+          const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * kKVTileBytes) >> 4);
+          uint32_t acc = (pv_started >> t) & 1;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(pa + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(va + kk * 2048, 8192, 1024);
-              umma_ss(d_tmem, ad, bd, idesc_pv, (pv_started[t] | kk) ? 1u : 0u);
-            }
-            pv_started[t] = 1;
-            umma_commit(&sm.pv_done[t]);
+          for (int kk = 0; kk < 8; ++kk) {
+            if (!((flag >> (kk >> 2)) & 1)) continue;
+            umma_ts(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + ((kk * 2048) >> 4),
+                    idesc_pv, acc);
+            acc = 1;
           }
-          umma_commit(&sm.v_empty[vs]);
-          if (++vs == kVStages) { vs = 0; vph ^= 1u; }
+          pv_started |= 1 << t;
+          umma_commit(&sm.pv_done[t]);
           return true;
         };
-        auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
-          const int act = ((mem & 3) ? 1 : 0) | ((mem & 12) ? 2 : 0);
+        auto finish_prev = [&]() -> bool {
+          int f1 = 0;
+          if (pend.act1) {
+            if (!mbar_wait_t(&sm.p_full[1], (pph >> 1) & 1u, wctx, pacc[2])) return false;
+            pph ^= 2u;
+            f1 = sm.pv_flag[1];
+          }
+          if (pend.f0 | f1) {
+            if (f1) {
+              if (!pend.v_waited) {
+                if (!mbar_wait_t(&sm.v_full[vs], vph, wctx, pacc[3])) return false;
+                tc_fence_after();
+              }
+              if (!issue_pv(1, f1)) return false;
+            }
+            umma_commit(&sm.v_empty[vs]);
+            if (++vs == kVStages) { vs = 0; vph ^= 1u; }
+          }
+          pend.valid = 0;
+          return true;
+        };
+        auto issue_qk = [&](int t, uint64_t kd) {
+          const uint64_t qd = qdesc0 + static_cast<uint64_t>((t * kQTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + t * 256, qd + off, kd + off, idesc_qk, kk ? 1u : 0u);
+          }
+          umma_commit(&sm.s_full[t]);
+        };
+        auto body = [&](int kt, bool is_col, int mem) -> bool {
+          const int act = (pf_tile_halves(mem, 0) ? 1 : 0) | (pf_tile_halves(mem, 1) ? 2 : 0);
           if (!mbar_wait_t(&sm.k_full[ks], kph, wctx, pacc[0])) return false;
           pacc[7] += 1;
           tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (!((act >> t) & 1)) continue;
-            const int bsel = sbuf[t];
-            if (!mbar_wait_t(&sm.s_empty[t][bsel], sph[t][bsel] ^ 1u, wctx, pacc[1])) return false;
-            sph[t][bsel] ^= 1u;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem + t * 256 + bsel * 64;
-            const uint32_t qa = smem_u32(sm.q[t]);
-            const uint32_t ka = smem_u32(sm.k[ks]);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-              umma_ss(d_tmem, ad, bd, idesc_qk, kk ? 1u : 0u);
-            }
-            umma_commit(&sm.s_full[t][bsel]);
-            sbuf[t] ^= 1;
-          }
+          const uint64_t kd = kdesc0 + static_cast<uint64_t>((ks * kKVTileBytes) >> 4);
+          if (act & 1) issue_qk(0, kd);
+          if (pend.valid && !finish_prev()) return false;
+          if (act & 2) issue_qk(1, kd);
           umma_commit(&sm.k_empty[ks]);
           if (++ks == kKStages) { ks = 0; kph ^= 1u; }
-          if (prev_act && !do_pv(prev_act)) return false;
-          prev_act = act;
+          int f0 = 0, v_waited = 0;
+          if (act & 1) {
+            if (!mbar_wait_t(&sm.p_full[0], pph & 1u, wctx, pacc[2])) return false;
+            pph ^= 1u;
+            f0 = sm.pv_flag[0];
+            if (f0) {
+              if (!mbar_wait_t(&sm.v_full[vs], vph, wctx, pacc[3])) return false;
+              tc_fence_after();
+              v_waited = 1;
+              if (!issue_pv(0, f0)) return false;
+            }
+          }
+          pend = {1, (act >> 1) & 1, f0, v_waited};
           return true;
         };
         ok = pf_for_each<has_cols>(sc, body);
-        if (ok && prev_act) ok = do_pv(prev_act);
+        if (ok && pend.valid) ok = finish_prev();
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!ofree_waited[t]) {
-            ok = mbar_wait(&sm.o_free[t], ofph[t] ^ 1u, wctx);
-            ofph[t] ^= 1u;
+          if (!((ofree_waited >> t) & 1)) {
+            ok = mbar_wait(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx);
+            ofph ^= 1u << t;
           }
         }
         umma_commit(&sm.q_empty);
         mbar_arrive(&sm.sched_empty[ub]);
       }
-      // make sure every issued tcgen05 op has finished before TMEM is freed
+      // every issued tcgen05 op must finish before TMEM is freed
       umma_commit(&sm.q_empty);
       mbar_wait_short(&sm.q_empty, (n & 1));
     }
@@ -553,12 +610,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 256;
     const int bar_id = 1 + t;
     const float NEG = -INFINITY;
-    int sbuf = 0;
-    uint32_t sphase = 0;  // bit b: phase of S buffer b
+    uint32_t sph = 0;
     int dslot = 0;
     uint32_t dph = 0;
     int dbuf = 0;
-    int pslot = 0;        // p_full / pv_flag ring slot of this tile
     uint32_t pv_total = 0;  // PVs issued for this tile so far (pv_done phases)
     bool ok = true;
     int n = 0;
@@ -569,14 +624,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!ok) break;
       const int my_valid = sc.seg_valid[seg];
       const int my_row = sc.seg_row0[seg] + (r & 63);
+      const bool row_ok = my_valid && my_row < p.Sq;
       float m_used = NEG, l = 0.f;
       int npv = 0;
-      auto body = [&](int item, int kt, bool is_col, int mem) -> bool {
-        const bool tile_act = (mem >> (2 * t)) & 3;
-        if (!tile_act) {
+      auto body = [&](int kt, bool is_col, int mem) -> bool {
+        const int tmask = pf_tile_halves(mem, t);
+        if (!tmask) {
           if (gated) {
-            if (tid == 128 + 128 * t) {
-              if (!mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2])) return false;
+            bool fail = false;
+            if (r == 0) fail = !mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2]);
+            // every wait result is agreed on before anyone leaves: the named
+            // barriers below must always see all 128 threads
+            if (named_bar_or(bar_id, 128, fail)) return false;
+            if (r == 0) {
               sm.dec_val[dslot][t] = 0;
               mbar_arrive(&sm.dec_full[dslot]);
             }
@@ -584,91 +644,106 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           return true;
         }
-        const bool seg_act = ((mem >> seg) & 1) && my_row < p.Sq;
-        if (!mbar_wait_t(&sm.s_full[t][sbuf], (sphase >> sbuf) & 1u, wctx, pacc[0])) return false;
-        sphase ^= 1u << sbuf;
+        const int segm = row_ok ? (mem >> (2 * seg)) & 3 : 0;
+        bool okw = mbar_wait_t(&sm.s_full[t], sph, wctx, pacc[0]);
+        // tcgen05.ld below is warp-collective: the warp leaves together
+        okw = __all_sync(0xffffffffu, okw);
+        if (!gated && !okw) return false;
+        sph ^= 1u;
         tc_fence_after();
-        float s[64];
-        tmem_ld64(lane_addr + sbuf * 64, s);
-        tc_fence_before();
-        mbar_arrive(&sm.s_empty[t][sbuf]);
-        sbuf ^= 1;
         pacc[5] += 1;
-        // ---- masks: row max over the visible keys of this tile
-        float rmax = NEG;
-        if (has_cols && is_col) {
+        // ---- pass 1: masks and per-half row maxima (one 64-column half at a time)
+        auto mask_half = [&](float* sh, int h) {
+          if (has_cols && is_col) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int e = kt * 64 + c;
-            bool vis = seg_act && e < sc.n_cols && ((sc.colmask[e] >> seg) & 1);
-            if (vis && p.causal) vis = sc.col[e] <= my_row + p.causal_off;
-            s[c] = vis ? s[c] : NEG;
+            for (int c = 0; c < 64; ++c) {
+              const int e = kt * 128 + 64 * h + c;
+              bool vis = ((segm >> h) & 1) && e < sc.n_cols && ((sc.colmask[e] >> seg) & 1);
+              if (vis && p.causal) vis = sc.col[e] <= my_row + p.causal_off;
+              sh[c] = vis ? sh[c] : NEG;
+            }
+          } else {
+            const int key0 = kt * 128 + 64 * h;
+            int lim = ((segm >> h) & 1) ? 64 : 0;
+            lim = min(lim, p.Sk - key0);
+            if (p.causal) lim = min(lim, my_row + p.causal_off - key0 + 1);
+            if (lim < 64) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c) sh[c] = (c < lim) ? sh[c] : NEG;
+            }
           }
-        } else {
-          // keys [key0, key0 + lim) of this tile are visible to the row
-          const int key0 = kt * 64;
-          int lim = seg_act ? 64 : 0;
-          lim = min(lim, p.Sk - key0);
-          if (p.causal) lim = min(lim, my_row + p.causal_off - key0 + 1);
-          if (lim < 64) {
+        };
+        float rm[2] = {NEG, NEG};
+        if (okw) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] = (c < lim) ? s[c] : NEG;
+          for (int h = 0; h < 2; ++h) {
+            float sh[64];
+            tmem_ld64(lane_addr + 64 * h, sh);
+            mask_half(sh, h);
+            float m4[4] = {NEG, NEG, NEG, NEG};
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sh[c]);
+            rm[h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           }
         }
-        {
-          float m4[4] = {NEG, NEG, NEG, NEG};
-#pragma unroll
-          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-          rmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        }
-        bool my_keep = seg_act;
-        bool tile_keep = true;
+        int my_keep = segm;
+        int flag = tmask;
         if (gated) {
           // exact block max of each 64 x 64 sub-tile (BSFA Figure 2a)
-          float wm = rmax;
-          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 16));
-          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 8));
-          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 4));
-          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 2));
-          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 1));
-          if (lane == 0) sm.red[t][dbuf][quarter] = wm;
-          named_bar_sync(bar_id, 128);
-          bool keep2[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float wm = rm[h];
+            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 16));
+            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 8));
+            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 4));
+            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 2));
+            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 1));
+            if (lane == 0) sm.red[t][dbuf][quarter][h] = wm;
+          }
+          bool fail = !okw;
+          if (r == 0 && !fail) fail = !mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2]);
+          if (named_bar_or(bar_id, 128, fail)) return false;
+          flag = 0;
+#pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int sgi = 2 * t + hh;
-            const float bmax = fmaxf(sm.red[t][dbuf][2 * hh], sm.red[t][dbuf][2 * hh + 1]);
-            const bool act = (mem >> sgi) & 1;
-            const float smax = bmax * p.scale;
-            const bool diag = kt == sc.seg_qb[sgi];
-            keep2[hh] = act && (diag || smax >= sc.seg_T[sgi]);
-            if (act && (r == 64 * hh)) {
-              const int64_t oi =
-                  ((static_cast<int64_t>(sc.b) * p.Hq + sc.seg_head[sgi]) * p.nqb +
-                   sc.seg_qb[sgi]) * p.nqb + kt;
-              if (p.smax_out) p.smax_out[oi] = smax;
-              if (p.keep_out) p.keep_out[oi] = keep2[hh] ? 1 : 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const bool act = (mem >> (2 * sgi + h)) & 1;
+              const float bmax = fmaxf(sm.red[t][dbuf][2 * hh][h], sm.red[t][dbuf][2 * hh + 1][h]);
+              const float smax = bmax * p.scale;
+              const int j = 2 * kt + h;
+              const bool keep = act && (j == sc.seg_qb[sgi] || smax >= sc.seg_T[sgi]);
+              if (keep) flag |= 1 << h;
+              if (hh == hseg) my_keep = (my_keep & ~(1 << h)) | ((keep && row_ok) ? 1 << h : 0);
+              if (act && r == 64 * hh + h) {
+                const int64_t oi =
+                    ((static_cast<int64_t>(sc.b) * p.Hq + sc.seg_head[sgi]) * p.nqb +
+                     sc.seg_qb[sgi]) * p.nqb + j;
+                if (p.smax_out) p.smax_out[oi] = smax;
+                if (p.keep_out) p.keep_out[oi] = keep ? 1 : 0;
+              }
             }
           }
           dbuf ^= 1;
-          my_keep = hseg ? keep2[1] : keep2[0];
-          tile_keep = keep2[0] || keep2[1];
           if (r == 0) {
-            if (!mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2])) return false;
-            sm.dec_val[dslot][t] = tile_keep ? 1 : 0;
+            sm.dec_val[dslot][t] = flag;
             mbar_arrive(&sm.dec_full[dslot]);
           }
           if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
         }
-        if (!tile_keep) {
-          if (r == 0) sm.pv_flag[t][pslot] = 0;
-          mbar_arrive(&sm.p_full[t][pslot]);
-          pslot ^= 1;
+        if (!flag) {
+          if (r == 0) sm.pv_flag[t] = 0;
+          mbar_arrive(&sm.p_full[t]);
           return true;
         }
-        // ---- online softmax (log2 domain, lazy rescale)
+        // ---- online softmax over the kept halves (log2 domain, lazy rescale)
+        float rmax = NEG;
+        if (my_keep & 1) rmax = rm[0];
+        if (my_keep & 2) rmax = fmaxf(rmax, rm[1]);
         float alpha = 1.f;
         bool resc = false;
-        if (my_keep && rmax != NEG) {
+        if (rmax != NEG) {
           const float mrow = rmax * p.scale_log2;
           if (mrow > m_used + 8.f) {
             alpha = ex2_approx(m_used - mrow);
@@ -677,50 +752,52 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
         const float mu = (m_used == NEG) ? 0.f : m_used;
-        uint32_t pk[32];
-        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (my_keep) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -mu));
-            const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -mu));
-            ps4[(c >> 1) & 3] += p0 + p1;
-            pk[c >> 1] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk[c] = 0u;
-        }
-        l = l * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
-        if (npv > 0) {
-          if (!mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1])) return false;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, resc)) {
-            pacc[6] += 1;
-            float ob[32];
+        // the commit behind s_full also covers the previous PV: O is stable here
+        if (npv > 0 && __any_sync(0xffffffffu, resc)) {
+          pacc[6] += 1;
+          float ob[32];
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              tmem_ld32(lane_addr + 128 + c * 32, ob);
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(lane_addr + 128 + c * 32, ob);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ob[i] *= alpha;
-              tmem_st32(lane_addr + 128 + c * 32, ob);
-            }
+            for (int i = 0; i < 32; ++i) ob[i] *= alpha;
+            tmem_st32(lane_addr + 128 + c * 32, ob);
           }
         }
-        // P row -> shared memory (K-major, 128B swizzle)
-        const uint32_t prow = smem_u32(sm.p[t]);
+        // ---- pass 2: P = exp2(s - m) per half, stored as bf16 pairs over the
+        // first 64 columns of S (half 0 -> columns 0..31, half 1 -> 32..63;
+        // half 1 is reloaded from columns 64..127, which P never overwrites)
+        float psum = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, cc)),
-                       "r"(pk[cc * 4]), "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]),
-                       "r"(pk[cc * 4 + 3])
-                       : "memory");
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+          const bool mine = (my_keep >> h) & 1;
+          // tcgen05.ld is warp-collective: reload when any lane of the warp
+          // keeps this half (rows differ in validity inside a ragged block)
+          if (__any_sync(0xffffffffu, mine)) {
+            float sh[64];
+            tmem_ld64(lane_addr + 64 * h, sh);
+            mask_half(sh, h);
+            const float base = mine ? mu : INFINITY;  // exp2(-inf) = 0 for lanes without it
+            float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float p0 = ex2_approx(fmaf(sh[c], p.scale_log2, -base));
+              const float p1 = ex2_approx(fmaf(sh[c + 1], p.scale_log2, -base));
+              ps4[(c >> 1) & 3] += p0 + p1;
+              pk[c >> 1] = pack_bf16x2(p0, p1);
+            }
+            psum += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pk[c] = 0u;
+          }
+          tmem_st32(lane_addr + 32 * h, reinterpret_cast<const float*>(pk));
         }
-        fence_proxy_async_smem();
+        l = l * alpha + psum;
         tc_fence_before();
-        if (r == 0) sm.pv_flag[t][pslot] = 1;
-        mbar_arrive(&sm.p_full[t][pslot]);
-        pslot ^= 1;
+        if (r == 0) sm.pv_flag[t] = flag;
+        mbar_arrive(&sm.p_full[t]);
         ++npv;
         ++pv_total;
         pacc[7] += 1;
@@ -729,11 +806,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       ok = pf_for_each<has_cols>(sc, body);
       if (!ok) break;
       // ---- epilogue: o = O / l, lse = ln(sum)
-      const bool store = my_valid && my_row < p.Sq;
+      const bool store = row_ok;
       const int head = sc.seg_head[seg];
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       if (npv > 0) {
-        if (!mbar_wait(&sm.pv_done[t], (pv_total - 1) & 1, wctx)) { ok = false; break; }
+        const bool okd = __all_sync(0xffffffffu,
+                                    mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1]));
+        if (!okd) { ok = false; break; }
         tc_fence_after();
         float ob[32];
 #pragma unroll 1
@@ -784,13 +863,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     else if (tid == 32) base = 16;     // MMA issuer
     else if (tid == 128) base = 24;    // softmax tile 0
     if (base >= 0) {
-      for (int i = 0; i < 7; ++i) atomicAdd(p.prof + base + i, pacc[i]);
-      atomicAdd(p.prof + base + 7, pacc[7]);
+      for (int i = 0; i < 8; ++i) atomicAdd(p.prof + base + i, pacc[i]);
       if (base == 24) atomicAdd(p.prof + 32, static_cast<unsigned long long>(clock64() - t_start));
     }
   }
 #else
   (void)t_start;
+  (void)pacc;
 #endif
   tc_fence_before();
   __syncthreads();
