@@ -254,18 +254,24 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
   p.o = static_cast<__nv_bfloat16*>(o.ptr); p.osb = o.sb; p.oss = o.ss; p.osh = o.sh;
   p.lse = lse;
   p.status = status;
-  CUtensorMap mKA, mVA, mKB, mVB;
   p.has_A = kA != nullptr;
   p.S_A = S_A;
   p.causal_A = causal_A;
   p.has_B = tb != nullptr;
+  auto set_src = [](const sbfa_t4* t, const __nv_bfloat16** ptr, int64_t* sb, int64_t* ss,
+                    int64_t* sh) {
+    *ptr = static_cast<const __nv_bfloat16*>(t->ptr);
+    *sb = t->sb;
+    *ss = t->ss;
+    *sh = t->sh;
+  };
   if (kA) {
-    SBFA_TRY(encode_bshd(&mKA, *kA, s->B, S_A, s->Hkv, 64));
-    SBFA_TRY(encode_bshd(&mVA, *vA, s->B, S_A, s->Hkv, 64));
+    set_src(kA, &p.kA, &p.kAsb, &p.kAss, &p.kAsh);
+    set_src(vA, &p.vA, &p.vAsb, &p.vAss, &p.vAsh);
   }
   if (tb) {
-    SBFA_TRY(encode_bshd(&mKB, *kB, s->B, s->Sk, s->Hkv, 64));
-    SBFA_TRY(encode_bshd(&mVB, *vB, s->B, s->Sk, s->Hkv, 64));
+    set_src(kB, &p.kB, &p.kBsb, &p.kBss, &p.kBsh);
+    set_src(vB, &p.vB, &p.vBsb, &p.vBss, &p.vBsh);
     p.S_B = s->Sk;
     p.kv_block = tb->kv_block;
     p.nmax = tb->nmax;
@@ -276,8 +282,6 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
   } else {
     p.S_B = 0; p.kv_block = 64; p.nmax = 0; p.n_kb = 0; p.idx = nullptr; p.tsb = p.tsh = 0;
   }
-  if (!kA) { mKA = mKB; mVA = mVB; }
-  if (!tb) { mKB = mKA; mVB = mVA; }
   const int grid = (grid_cap > 0 && grid_cap < di.sms) ? grid_cap : di.sms;
   if (ws) {
     const int tpairs = ticket_pairs > npairs ? ticket_pairs : npairs;
@@ -306,7 +310,7 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr_set[dev] = true;
   }
-  sbfa::decode_kernel<<<grid, sbfa::kDecThreads, smem, stream>>>(mKA, mVA, mKB, mVB, p);
+  sbfa::decode_kernel<<<grid, sbfa::kDecThreads, smem, stream>>>(p);
   SBFA_CUDA(cudaGetLastError());
   return SBFA_OK;
 }
