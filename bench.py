@@ -440,8 +440,17 @@ def main():
     import block_sparse_flashattention_sbfa_b200 as sb
 
     l2 = torch.cuda.get_device_properties(dist.local).L2_cache_size
-    flush_buf = torch.empty(max(4 * l2, 512 << 20), dtype=torch.uint8, device="cuda")
-    flush = lambda: flush_buf.fill_(1)  # noqa: E731
+    # L2 flush: write a buffer of 4x L2, then read another of 4x L2, so that
+    # the cache holds clean lines of neither input (a write-only flush leaves
+    # L2 full of dirty lines whose write-back would be charged to the next
+    # kernel).
+    nfl = max(4 * l2, 512 << 20)
+    flush_buf = torch.empty(nfl, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(nfl // 4, dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1)
+        flush_rd.sum()
 
     clocks = ClockSampler(dist.local).start()
     dec = bench_decode(torch, sb, dist, args, flush, peaks)
@@ -470,7 +479,7 @@ def main():
                                "D=128 bs=128, dense last 2048 + 32 missed blocks, fused "
                                "split-KV kernel", "global_batch": 8 * dist.world,
                    "seq_len": 32768, "parallelism": f"replicas x{dist.world}",
-                   "l2": "flushed before every step (4x L2 write), outside the timed events"},
+                   "l2": "flushed before every step (4x L2 write, then 4x L2 read), outside the timed events"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": ncu_traffic("decode_kernel"), "peak_kind": peak_kind,

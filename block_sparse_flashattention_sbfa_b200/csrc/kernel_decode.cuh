@@ -2,18 +2,26 @@
 // README, Usage 2) and short-query block-table attention, fused with the LSE
 // combine of the per-CTA pieces.
 //
-// Work: for every (batch b, kv-head g) pair the key set is a list of 64-key
-// chunks -- the dense source A (k_spec/v_spec) cut into chunks, followed by
-// the listed blocks of source B (k/v).  The chunks of all pairs are laid end
-// to end and every CTA of the persistent grid takes an equal contiguous
-// range of them (no load imbalance whatever the per-pair counts).  A CTA
-// streams its chunks through a TMA pipeline; four consumer warps each take 16
-// keys of a chunk and run QK^T and PV on mma.sync (the M = 16 tile carries
-// the <= 16 query rows of the pair: Sq positions x G query heads).  At the end
-// of its part of a pair the CTA merges its warps' running (m, l, O) and either
-// writes the final row (the pair lies wholly inside the CTA's range) or an
-// fp32 partial; the last CTA to finish a pair (atomic ticket) merges the
-// partials with the LSE combine and resets the ticket.
+// Work layout: every (batch b, kv-head g) pair owns a fixed run of `pp`
+// chunk slots of 64 keys -- the dense source A (k_spec/v_spec) cut into
+// chunks, then kv_block/64 slots per table entry of source B (k/v).  The
+// slots of all pairs are laid end to end and CTA c of the persistent grid
+// takes the contiguous range [total*c/grid, total*(c+1)/grid): the split is
+// known at launch, so no CTA scans the table before streaming.  A table
+// entry that is padding (< 0) leaves its slots empty: they cost no load.
+//
+// Inside a CTA two groups of four warps take alternate chunks; each warp
+// owns a 16-key slice of its group's chunks and streams the K and V rows of
+// its slices into a private three-stage cp.async ring (16-byte copies, zero
+// fill past the end), then runs QK^T and PV on mma.sync m16n8k16 (the M = 16
+// tile carries the <= 16 query rows of a pair: Sq positions x G query heads).
+// At the end of its part of a pair the CTA merges its warps' running
+// (m, l, O) and writes either the final row (the pair lies wholly inside its
+// range) or an fp32 partial.  A shared pair is finished by whichever CTA
+// takes the last ticket: tickets are taken right after each partial is
+// written but read only when the CTA has streamed its whole range, so no
+// warp waits on another CTA's progress; that CTA merges all partials with
+// the LSE combine and resets the ticket.
 #pragma once
 
 #include "sbfa_ptx.cuh"
@@ -23,18 +31,15 @@ namespace sbfa {
 constexpr int kDecChunk = 64;
 constexpr int kDecGroupWarps = 4;                        // warps per consumer group
 constexpr int kDecGroups = 2;                            // groups take alternate chunks
-constexpr int kDecGroupThreads = kDecGroupWarps * 32;
-constexpr int kDecThreads = kDecGroups * kDecGroupThreads;
-constexpr int kDecWarpStages = 2;                        // cp.async double buffer per warp
+constexpr int kDecWarps = kDecGroups * kDecGroupWarps;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecWarpStages = 3;                        // cp.async ring depth per warp
 constexpr int kDecSliceKeys = 16;                        // keys of a chunk one warp owns
 constexpr int kDecSliceBytes = 2 * kDecSliceKeys * 128 * 2;  // K + V slice, bf16
 constexpr int kDecMaxPairs = 4096;
 constexpr int kDecMaxEntries = 1024;
-constexpr int kDecMaxList = 2048;                        // chunks per window
-constexpr int kDecMaxPieces = 256;                       // pair pieces per window
 constexpr int kDecRows = 16;
 constexpr int kDecD = 128;
-constexpr int kDecStageBytes = 2 * kDecChunk * kDecD * 2;  // K + V, bf16
 
 struct DecodeParams {
   int B, Sq, Hq, Hkv, G, rows;
@@ -62,27 +67,13 @@ struct DecodeParams {
   int* status;
 };
 
-struct DecPiece {
-  int pr, kbeg, kend, flags;  // list positions [kbeg, kend); flags: 1 = the CTA's
-                              // part of pair pr starts in this window, 2 = ends in it
-  int c_from;                 // pair-local chunk index of list position kbeg
-};
-
 struct DecSmem {
-  alignas(1024) uint8_t slice[kDecGroups * kDecGroupWarps][kDecWarpStages][kDecSliceBytes];
+  alignas(1024) uint8_t slice[kDecWarps][kDecWarpStages][kDecSliceBytes];
+  float ow[kDecGroupWarps][kDecRows][kDecD];
   float mw[kDecGroupWarps][kDecRows];
   float lw[kDecGroupWarps][kDecRows];
-  float ow[kDecGroupWarps][kDecRows][kDecD];
-  int prefix[kDecMaxPairs + 1];
-  int entries[kDecMaxEntries];
-  int2 chunk[kDecMaxList];  // {key0, nkeys | src << 8}
-  DecPiece piece[kDecMaxPieces];
-  int n_pieces, n_list;
-  int64_t next_x;           // window builder cursor (next global chunk of this CTA)
-  int next_pr;
-  int is_last;
-  int n_split;
-  int split_pr[2];  // pairs this CTA shares with others (stream-K: first and last)
+  int2 meta[kDecWarps][kDecWarpStages];  // slice in each stage: {key0, nk | src << 7 | pr << 8}
+  int last[2];                           // this CTA finishes shared pair 0 / 1
 };
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decode shared memory exceeds 227 KB");
@@ -95,30 +86,12 @@ __device__ __forceinline__ int64_t dec_range_lo(int c, int64_t total, int grid) 
   return (total * c) / grid;
 }
 
-// CTA whose range holds global chunk x.
+// CTA whose range holds global slot x.
 __device__ __forceinline__ int dec_cta_of(int64_t x, int64_t total, int grid) {
   int c = static_cast<int>((x * grid) / total);
   while (c + 1 < grid && dec_range_lo(c + 1, total, grid) <= x) ++c;
   while (c > 0 && dec_range_lo(c, total, grid) > x) --c;
   return c;
-}
-
-// Number of CTAs in [c_first, c_last] whose chunk range is not empty.
-__device__ __forceinline__ int dec_nonempty_ctas(int c_first, int c_last, int64_t total, int grid) {
-  int n = 0;
-  for (int c = c_first; c <= c_last; ++c)
-    n += dec_range_lo(c, total, grid) < dec_range_lo(c + 1, total, grid) ? 1 : 0;
-  return n;
-}
-
-// Pair holding global chunk x (prefix is non-decreasing, prefix[n] = total).
-__device__ __forceinline__ int dec_pair_of(const int* prefix, int npairs, int64_t x) {
-  int lo = 0, hi = npairs;  // prefix[lo] <= x < prefix[hi]
-  while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
-    if (prefix[mid] <= x) lo = mid; else hi = mid;
-  }
-  return lo;
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0,
@@ -135,14 +108,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
-}
-
-// Address of bf16 element (key, d) of a 64 x 128 tile stored as two
-// 128B-swizzled halves of 64 columns.
-__device__ __forceinline__ uint32_t dec_elem_addr(uint32_t base, int key, int d) {
-  const int half = d >> 6;
-  const int byte = (d & 63) * 2;
-  return base + half * 8192 + sw128_off(key, byte >> 4) + (byte & 15);
 }
 
 // Address of bf16 element (key, d) of a 16-key slice stored as two
@@ -168,281 +133,183 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   const int npairs = p.B * p.Hkv;
   const int grid = gridDim.x;
   const int cta = blockIdx.x;
+  const float NEG = -INFINITY;
   const int nA = p.has_A ? (p.S_A + kDecChunk - 1) / kDecChunk : 0;
   const int cpe = dec_chunks_per_entry(p.kv_block);
-  const int keys_per_entry_chunk = p.kv_block < kDecChunk ? p.kv_block : kDecChunk;
+  const int kpc = p.kv_block < kDecChunk ? p.kv_block : kDecChunk;  // keys per B slot
+  const int pp = nA + (p.has_B ? p.nmax * cpe : 0);                  // slots per pair
 
-  // ---- per-pair chunk counts and their prefix sum (every CTA computes the same)
-  for (int pr = tid; pr < npairs; pr += kDecThreads) sm.prefix[pr + 1] = nA;
-  __syncthreads();
-  if (p.has_B) {
-    const int n_ent = npairs * p.nmax;
-    for (int base = 0; base < n_ent; base += 4 * kDecThreads) {
-      int jv[4], pv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = base + u * kDecThreads + tid;
-        pv[u] = -1;
-        jv[u] = -1;
-        if (e < n_ent) {
-          const int pr = e / p.nmax, n = e % p.nmax;
-          pv[u] = pr;
-          jv[u] = __ldg(p.idx + (pr / p.Hkv) * p.tsb + (pr % p.Hkv) * p.tsh + n);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (pv[u] < 0) continue;
-        if (jv[u] >= 0 && jv[u] < p.n_kb) atomicAdd(&sm.prefix[pv[u] + 1], cpe);
-        else if (jv[u] >= p.n_kb && cta == 0) report(p.status, kDevBadIndex);
+  if (pp == 0) {  // no key at all: every row is (o = 0, lse = -inf)
+    for (int pr = cta; pr < npairs; pr += grid) {
+      const int b = pr / p.Hkv, g = pr % p.Hkv;
+      for (int e = tid; e < p.rows * kDecD; e += kDecThreads) {
+        const int rr = e / kDecD, d = e % kDecD;
+        const int sq = rr / p.G, h = g * p.G + rr % p.G;
+        p.o[b * p.osb + sq * p.oss + h * p.osh + d] = __float2bfloat16(0.f);
+        if (d == 0) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.Sq + sq] = NEG;
       }
     }
+    return;
   }
-  __syncthreads();
-  if (warp == 0) {
-    int carry = 0;
-    if (lane == 0) sm.prefix[0] = 0;
-    for (int base = 0; base < npairs; base += 32) {
-      int v = (base + lane < npairs) ? sm.prefix[base + lane + 1] : 0;
-      for (int off = 1; off < 32; off <<= 1) {
-        int t = __shfl_up_sync(0xffffffffu, v, off);
-        if (lane >= off) v += t;
-      }
-      if (base + lane < npairs) sm.prefix[base + lane + 1] = v + carry;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-  }
-  __syncthreads();
-  const int64_t total = sm.prefix[npairs];
-
-  // Pairs with no key at all: write the neutral result (o = 0, lse = -inf).
-  for (int pr = cta; pr < npairs; pr += grid) {
-    if (sm.prefix[pr + 1] != sm.prefix[pr]) continue;
-    const int b = pr / p.Hkv, g = pr % p.Hkv;
-    for (int e = tid; e < p.rows * kDecD; e += kDecThreads) {
-      const int rr = e / kDecD, d = e % kDecD;
-      const int sq = rr / p.G, h = g * p.G + rr % p.G;
-      p.o[b * p.osb + sq * p.oss + h * p.osh + d] = __float2bfloat16(0.f);
-      if (d == 0) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.Sq + sq] = -INFINITY;
-    }
-  }
-  if (total == 0) return;
-  // This CTA's chunks: stream-K = the contiguous global range [lo, hi); pair
+  const int64_t total = static_cast<int64_t>(npairs) * pp;
+  // This CTA's slot sequence: stream-K = the global range [lo, hi); pair
   // mode = whole pairs cta, cta + grid, ...
-  const int64_t lo = p.pair_mode ? 0 : dec_range_lo(cta, total, grid);
-  const int64_t hi = p.pair_mode ? total : dec_range_lo(cta + 1, total, grid);
-  if (lo >= hi) return;
-  const int first_pair = p.pair_mode ? cta : dec_pair_of(sm.prefix, npairs, lo);
-  const int pair_step = p.pair_mode ? grid : 1;
+  int64_t lo = 0, hi = 0, N;
+  int n_pieces;
+  if (p.pair_mode) {
+    n_pieces = cta < npairs ? (npairs - cta + grid - 1) / grid : 0;
+    N = static_cast<int64_t>(n_pieces) * pp;
+  } else {
+    lo = dec_range_lo(cta, total, grid);
+    hi = dec_range_lo(cta + 1, total, grid);
+    n_pieces = hi > lo ? static_cast<int>((hi - 1) / pp - lo / pp + 1) : 0;
+    N = hi - lo;
+  }
+  if (N == 0) return;
+  // global slot of sequence position n
+  auto seq_x = [&](int64_t n) -> int64_t {
+    if (p.pair_mode) return (cta + (n / pp) * grid) * static_cast<int64_t>(pp) + n % pp;
+    return lo + n;
+  };
 
   const int grp = warp / kDecGroupWarps, wg = warp % kDecGroupWarps;
-  const int gt = tid % kDecGroupThreads;  // thread index inside the group
   const int gq = lane >> 2, cq = lane & 3;
-  const float NEG = -INFINITY;
-  if (tid == 0) {
-    sm.next_pr = first_pair;
-    sm.next_x = 0;  // chunks of pair next_pr already handed out (pair-local)
-    sm.n_split = 0;
-  }
-  __syncthreads();
+  const int n_mine = static_cast<int>((N - grp + 1) / 2);  // positions grp, grp + 2, ...
+  const int kw = wg * kDecSliceKeys;
 
-  // running state of the piece in progress (persists across windows)
+  // Slot metadata of this warp's chunks j in [32 w, 32 w + 32), lane j % 32.
+  int mkey = 0, minfo = 0;
+  auto load_meta = [&](int win) {
+    const int j = win * 32 + lane;
+    int key0 = 0, info = 0;
+    if (j < n_mine) {
+      const int64_t x = seq_x(grp + 2 * static_cast<int64_t>(j));
+      const int pr = static_cast<int>(x / pp), c = static_cast<int>(x % pp);
+      int nk = 0, src = 0;
+      if (c < nA) {
+        key0 = c * kDecChunk;
+        nk = min(kDecChunk, p.S_A - key0);
+      } else {
+        src = 1;
+        const int e = (c - nA) / cpe, sub = (c - nA) % cpe;
+        const int b = pr / p.Hkv, g = pr % p.Hkv;
+        const int jb = __ldg(p.idx + b * p.tsb + g * p.tsh + e);
+        if (jb >= 0 && jb < p.n_kb) {
+          key0 = jb * p.kv_block + sub * kDecChunk;
+          nk = max(min(kpc, p.S_B - key0), 0);
+        } else if (jb >= p.n_kb) {
+          report(p.status, kDevBadIndex);
+        }
+      }
+      info = nk | (src << 7) | (pr << 8);
+    }
+    mkey = key0;
+    minfo = info;
+  };
+
+  // Stream chunk j's slice of this warp into ring stage j % kDecWarpStages.
+  // One commit group per call (empty past the end), so that "all but the
+  // newest kDecWarpStages - 1 groups" is always the group of the oldest stage.
+  auto issue = [&](int j) {
+    const int stage = j % kDecWarpStages;
+    if (j < n_mine) {
+      if ((j & 31) == 0 && j > 0) load_meta(j >> 5);
+      const int key0 = __shfl_sync(0xffffffffu, mkey, j & 31);
+      const int info = __shfl_sync(0xffffffffu, minfo, j & 31);
+      if (lane == 0) sm.meta[warp][stage] = make_int2(key0, info);
+      const int nk = info & 0x7f, src = (info >> 7) & 1, pr = info >> 8;
+      if (nk > kw) {
+        const int b = pr / p.Hkv, g = pr % p.Hkv;
+        const __nv_bfloat16* krow0 =
+            src ? p.kB + b * p.kBsb + g * p.kBsh : p.kA + b * p.kAsb + g * p.kAsh;
+        const __nv_bfloat16* vrow0 =
+            src ? p.vB + b * p.vBsb + g * p.vBsh : p.vA + b * p.vAsb + g * p.vAsh;
+        const int64_t kro = src ? p.kBss : p.kAss, vro = src ? p.vBss : p.vAss;
+        const uint32_t kdst = smem_u32(sm.slice[warp][stage]);
+#pragma unroll
+        for (int it = 0; it < kDecSliceKeys * 16 / 32; ++it) {
+          const int e = lane + it * 32;
+          const int r = e >> 4, ch = e & 15;
+          const uint32_t off = (ch >> 3) * (kDecSliceKeys * 128) + sw128_off(r, ch & 7);
+          const bool valid = kw + r < nk;
+          const int64_t row = valid ? key0 + kw + r : 0;
+          const uint32_t bytes = valid ? 16u : 0u;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(kdst + off),
+                       "l"(krow0 + row * kro + ch * 8), "r"(bytes)
+                       : "memory");
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                           kdst + kDecSliceBytes / 2 + off),
+                       "l"(vrow0 + row * vro + ch * 8), "r"(bytes)
+                       : "memory");
+        }
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  load_meta(0);
+#pragma unroll
+  for (int s = 0; s < kDecWarpStages; ++s) issue(s);
+
+  // running state of the piece in progress
   uint32_t qa[8][4];
   float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
   float oacc[16][4];
   bool v0 = false, v1 = false;
   int lim0 = -1, lim1 = -1;
+  int ticket0 = 0, ticket1 = 0;  // thread 0: tickets of the shared first / last pair
+  int j = 0;
 
-  // A pair shared with other CTAs: after this CTA's partial is written, the
-  // last CTA to finish the pair merges all partials with the LSE combine.
-  auto finish_split = [&](const int pr) {
-    __threadfence();
-    __syncthreads();
-    const int d = tid % kDecD;
-    const int rpar = tid / kDecD;
+  for (int pi = 0; pi < n_pieces; ++pi) {
+    int pr;
+    int64_t nb, ne;
+    bool whole;
+    if (p.pair_mode) {
+      pr = cta + pi * grid;
+      nb = static_cast<int64_t>(pi) * pp;
+      ne = nb + pp;
+      whole = true;
+    } else {
+      pr = static_cast<int>(lo / pp) + pi;
+      const int64_t a = static_cast<int64_t>(pr) * pp, e = a + pp;
+      nb = (a > lo ? a : lo) - lo;
+      ne = (e < hi ? e : hi) - lo;
+      whole = a >= lo && e <= hi;
+    }
     const int b = pr / p.Hkv, g = pr % p.Hkv;
-    const int64_t pbeg = sm.prefix[pr], pend = sm.prefix[pr + 1];
-    const int c_first = dec_cta_of(pbeg, total, grid);
-    const int c_last = dec_cta_of(pend - 1, total, grid);
-    if (tid == 0) {
-      const int old = atomicAdd(&p.ws_ticket[pr], 1);
-      sm.is_last = (old == dec_nonempty_ctas(c_first, c_last, total, grid) - 1) ? 1 : 0;
-      if (sm.is_last) __threadfence();
-    }
-    __syncthreads();
-    if (sm.is_last) {
-      for (int rr = rpar; rr < p.rows; rr += 2) {
-        float M = -INFINITY;
-        for (int cc = c_first; cc <= c_last; ++cc) {
-          if (dec_range_lo(cc, total, grid) == dec_range_lo(cc + 1, total, grid)) continue;
-          const int fp = dec_pair_of(sm.prefix, npairs, dec_range_lo(cc, total, grid));
-          const int sl = (fp == pr) ? 2 * cc : 2 * cc + 1;
-          M = fmaxf(M, __ldcg(&p.ws_lse[sl * kDecRows + rr]));
-        }
-        const float Mn = (M == -INFINITY) ? 0.f : M;
-        float W = 0.f, acc = 0.f;
-        for (int cc = c_first; cc <= c_last; ++cc) {
-          if (dec_range_lo(cc, total, grid) == dec_range_lo(cc + 1, total, grid)) continue;
-          const int fp = dec_pair_of(sm.prefix, npairs, dec_range_lo(cc, total, grid));
-          const int sl = (fp == pr) ? 2 * cc : 2 * cc + 1;
-          const float lv = __ldcg(&p.ws_lse[sl * kDecRows + rr]);
-          const float wt = (lv == -INFINITY) ? 0.f : __expf(lv - Mn);
-          W += wt;
-          acc += wt * __ldcg(&p.ws_part[(static_cast<int64_t>(sl) * kDecRows + rr) * kDecD + d]);
-        }
-        const int sq = rr / p.G, h = g * p.G + rr % p.G;
-        p.o[b * p.osb + sq * p.oss + h * p.osh + d] = __float2bfloat16(W > 0.f ? acc / W : 0.f);
-        if (d == 0)
-          p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.Sq + sq] = W > 0.f ? Mn + __logf(W) : -INFINITY;
-      }
-      if (tid == 0) p.ws_ticket[pr] = 0;
-    }
-    __syncthreads();
-  };
-
-  while (true) {
-    // ================= build the next window of chunks =================
-    if (tid == 0) {
-      int np = 0, nl = 0;
-      int pr = sm.next_pr;
-      int64_t used = sm.next_x;
-      while (pr < npairs && np < kDecMaxPieces && nl < kDecMaxList) {
-        const int64_t pbeg = sm.prefix[pr], pend = sm.prefix[pr + 1];
-        if (pbeg >= hi) { pr = npairs; break; }
-        const int64_t c0 = (lo > pbeg ? lo : pbeg) - pbeg;
-        const int64_t c1 = (hi < pend ? hi : pend) - pbeg;
-        if (c1 <= c0) { pr += pair_step; used = 0; continue; }
-        const int64_t from = c0 + used;
-        const int64_t take = min(static_cast<int64_t>(kDecMaxList - nl), c1 - from);
-        DecPiece pc;
-        pc.pr = pr;
-        pc.kbeg = nl;
-        pc.kend = nl + static_cast<int>(take);
-        pc.flags = (used == 0 ? 1 : 0) | (from + take == c1 ? 2 : 0);
-        pc.c_from = static_cast<int>(from);
-        sm.piece[np++] = pc;
-        nl += static_cast<int>(take);
-        if (from + take == c1) { pr += pair_step; used = 0; }
-        else used += take;
-      }
-      sm.n_pieces = np;
-      sm.n_list = nl;
-      sm.next_pr = pr;
-      sm.next_x = used;
-    }
-    __syncthreads();
-    const int n_pieces = sm.n_pieces, n_list = sm.n_list;
-    if (n_list == 0) break;
-    // chunk metadata of every list position; a piece's valid table entries
-    // are compacted first (in table order)
-    for (int pi = 0; pi < n_pieces; ++pi) {
-      const DecPiece pc = sm.piece[pi];
-      const int b = pc.pr / p.Hkv, g = pc.pr % p.Hkv;
-      if (p.has_B && warp == 0) {
-        const int* row = p.idx + b * p.tsb + g * p.tsh;
-        int nv = 0;
-        for (int base = 0; base < p.nmax; base += 32) {
-          const int n = base + lane;
-          const int j = n < p.nmax ? __ldg(row + n) : -1;
-          const bool valid = j >= 0 && j < p.n_kb;
-          const uint32_t bal = __ballot_sync(0xffffffffu, valid);
-          if (valid) sm.entries[nv + __popc(bal & ((1u << lane) - 1u))] = j;
-          nv += __popc(bal);
-        }
-      }
-      __syncthreads();
-      for (int k = pc.kbeg + tid; k < pc.kend; k += kDecThreads) {
-        const int c = pc.c_from + (k - pc.kbeg);
-        int src, key0, nk;
-        if (c < nA) {
-          src = 0;
-          key0 = c * kDecChunk;
-          nk = min(kDecChunk, p.S_A - key0);
-        } else {
-          const int e = (c - nA) / cpe, sub = (c - nA) % cpe;
-          src = 1;
-          key0 = sm.entries[e] * p.kv_block + sub * kDecChunk;
-          nk = min(keys_per_entry_chunk, p.S_B - key0);
-        }
-        nk = max(nk, 0);
-        sm.chunk[k] = make_int2(key0, nk | (src << 8) | (pi << 16));
-      }
-      __syncthreads();
-    }
-
-    // ================= consume: two groups, cp.async double buffer =================
-    const int n_mine = (n_list - grp + 1) / 2;  // list positions grp, grp + 2, ...
-    // Each warp streams its own 16-key slice of its group's chunks through a
-    // private double buffer: it waits only for its own copies (no barrier
-    // with other warps), so warps progress independently.
-    const int kw = wg * kDecSliceKeys;
-    auto issue = [&](int j) {
-      const int k = grp + 2 * j;
-      const int2 ci = sm.chunk[k];
-      const int key0 = ci.x, nk = ci.y & 0xff, src = (ci.y >> 8) & 1;
-      const int pr = sm.piece[ci.y >> 16].pr;
-      const int b = pr / p.Hkv, g = pr % p.Hkv;
-      const __nv_bfloat16* krow0 =
-          src ? p.kB + b * p.kBsb + g * p.kBsh : p.kA + b * p.kAsb + g * p.kAsh;
-      const __nv_bfloat16* vrow0 =
-          src ? p.vB + b * p.vBsb + g * p.vBsh : p.vA + b * p.vAsb + g * p.vAsh;
-      const int64_t kro = src ? p.kBss : p.kAss, vro = src ? p.vBss : p.vAss;
-      const uint32_t kdst = smem_u32(sm.slice[warp][j & 1]);
+    {
+      // Q fragments (A operand, 16 rows x 128) and per-row causal limits
+      const int r0 = gq, r1 = gq + 8;
+      v0 = r0 < p.rows;
+      v1 = r1 < p.rows;
+      lim0 = v0 ? r0 / p.G + (p.S_A - p.Sq) : -1;
+      lim1 = v1 ? r1 / p.G + (p.S_A - p.Sq) : -1;
+      const __nv_bfloat16* q0 =
+          v0 ? p.q + b * p.qsb + (r0 / p.G) * p.qss + (g * p.G + r0 % p.G) * p.qsh : nullptr;
+      const __nv_bfloat16* q1 =
+          v1 ? p.q + b * p.qsb + (r1 / p.G) * p.qss + (g * p.G + r1 % p.G) * p.qsh : nullptr;
 #pragma unroll
-      for (int it = 0; it < kDecSliceKeys * 16 / 32; ++it) {
-        const int e = lane + it * 32;
-        const int r = e >> 4, ch = e & 15;
-        const uint32_t off = (ch >> 3) * (kDecSliceKeys * 128) + sw128_off(r, ch & 7);
-        const bool valid = kw + r < nk;
-        const int64_t row = valid ? key0 + kw + r : 0;
-        const uint32_t bytes = valid ? 16u : 0u;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(kdst + off),
-                     "l"(krow0 + row * kro + ch * 8), "r"(bytes)
-                     : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
-                         kdst + kDecSliceBytes / 2 + off),
-                     "l"(vrow0 + row * vro + ch * 8), "r"(bytes)
-                     : "memory");
+      for (int ks = 0; ks < 8; ++ks) {
+        const int d = ks * 16 + 2 * cq;
+        qa[ks][0] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d)) : 0u;
+        qa[ks][1] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d)) : 0u;
+        qa[ks][2] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d + 8)) : 0u;
+        qa[ks][3] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d + 8)) : 0u;
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    if (n_mine > 0) issue(0);
-    if (n_mine > 1) issue(1);
-    int jc = 0;
-    for (int pi = 0; pi < n_pieces; ++pi) {
-      const DecPiece pc = sm.piece[pi];
-      const int b = pc.pr / p.Hkv, g = pc.pr % p.Hkv;
-      if (pc.flags & 1) {
-        // Q fragments (A operand, 16 rows x 128) and per-row limits for this pair
-        const int r0 = gq, r1 = gq + 8;
-        v0 = r0 < p.rows;
-        v1 = r1 < p.rows;
-        lim0 = v0 ? r0 / p.G + (p.S_A - p.Sq) : -1;
-        lim1 = v1 ? r1 / p.G + (p.S_A - p.Sq) : -1;
-        const __nv_bfloat16* q0 =
-            v0 ? p.q + b * p.qsb + (r0 / p.G) * p.qss + (g * p.G + r0 % p.G) * p.qsh : nullptr;
-        const __nv_bfloat16* q1 =
-            v1 ? p.q + b * p.qsb + (r1 / p.G) * p.qss + (g * p.G + r1 % p.G) * p.qsh : nullptr;
+      m0 = m1 = NEG;
+      l0 = l1 = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const int d = ks * 16 + 2 * cq;
-          qa[ks][0] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d)) : 0u;
-          qa[ks][1] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d)) : 0u;
-          qa[ks][2] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d + 8)) : 0u;
-          qa[ks][3] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d + 8)) : 0u;
-        }
-        m0 = m1 = NEG;
-        l0 = l1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-      }
-      for (; jc < n_mine && grp + 2 * jc < pc.kend; ++jc) {
-        if (jc + 1 < n_mine) asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncwarp();  // this warp's copies are in and visible to all its lanes
-        const int2 ci = sm.chunk[grp + 2 * jc];
-        const int key0 = ci.x, nkeys = ci.y & 0xff, src = (ci.y >> 8) & 1;
-        const uint32_t kbase = smem_u32(sm.slice[warp][jc & 1]);
+      for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+    }
+    const int j_end = static_cast<int>((ne - grp + 1) / 2);  // chunks with grp + 2 j < ne
+    for (; j < j_end; ++j) {
+      asm volatile("cp.async.wait_group %0;" ::"n"(kDecWarpStages - 1) : "memory");
+      __syncwarp();  // this warp's copies are in and visible to all its lanes
+      const int stage = j % kDecWarpStages;
+      const int2 mt = sm.meta[warp][stage];
+      const int key0 = mt.x, nkeys = mt.y & 0x7f, src = (mt.y >> 7) & 1;
+      if (nkeys > kw) {
+        const uint32_t kbase = smem_u32(sm.slice[warp][stage]);
         const uint32_t vbase = kbase + kDecSliceBytes / 2;
         float s[2][4];
 #pragma unroll
@@ -524,73 +391,71 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
             mma_bf16_16816(oacc[2 * dt2 + 1], pa, x2, x3);
           }
         }
-        __syncwarp();  // every lane is done with the buffer: refill it
-        if (jc + 2 < n_mine) issue(jc + 2);
       }
-      if (!(pc.flags & 2)) continue;  // the pair continues in the next window
-      // ---- merge the eight warps' states for this pair
-      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      // (1) group 1 publishes its state, group 0 folds it into its registers
-      if (grp == 1) {
-        if (cq == 0) {
-          sm.mw[wg][gq] = m0; sm.mw[wg][gq + 8] = m1;
-          sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
-        }
+      __syncwarp();  // every lane is done with the stage: refill it
+      issue(j + kDecWarpStages);
+    }
+
+    // ---- merge the eight warps' states for this pair
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    // (1) group 1 publishes its state, group 0 folds it into its registers
+    if (grp == 1) {
+      if (cq == 0) {
+        sm.mw[wg][gq] = m0; sm.mw[wg][gq + 8] = m1;
+        sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
+      }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int d = i * 8 + 2 * cq;
-          *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
-          *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
-        }
+      for (int i = 0; i < 16; ++i) {
+        const int d = i * 8 + 2 * cq;
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
       }
-      __syncthreads();
-      if (grp == 0) {
-        const float om0 = sm.mw[wg][gq], om1 = sm.mw[wg][gq + 8];
-        const float M0 = fmaxf(m0, om0), M1 = fmaxf(m1, om1);
-        const float Mu0 = (M0 == NEG) ? 0.f : M0, Mu1 = (M1 == NEG) ? 0.f : M1;
-        const float a0 = ex2_approx(m0 - Mu0), b0 = ex2_approx(om0 - Mu0);
-        const float a1 = ex2_approx(m1 - Mu1), b1 = ex2_approx(om1 - Mu1);
-        l0 = a0 * l0 + b0 * sm.lw[wg][gq];
-        l1 = a1 * l1 + b1 * sm.lw[wg][gq + 8];
-        m0 = M0;
-        m1 = M1;
+    }
+    __syncthreads();
+    if (grp == 0) {
+      const float om0 = sm.mw[wg][gq], om1 = sm.mw[wg][gq + 8];
+      const float M0 = fmaxf(m0, om0), M1 = fmaxf(m1, om1);
+      const float Mu0 = (M0 == NEG) ? 0.f : M0, Mu1 = (M1 == NEG) ? 0.f : M1;
+      const float a0 = ex2_approx(m0 - Mu0), b0 = ex2_approx(om0 - Mu0);
+      const float a1 = ex2_approx(m1 - Mu1), b1 = ex2_approx(om1 - Mu1);
+      l0 = a0 * l0 + b0 * sm.lw[wg][gq];
+      l1 = a1 * l1 + b1 * sm.lw[wg][gq + 8];
+      m0 = M0;
+      m1 = M1;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int d = i * 8 + 2 * cq;
-          const float2 x = *reinterpret_cast<const float2*>(&sm.ow[wg][gq][d]);
-          const float2 y = *reinterpret_cast<const float2*>(&sm.ow[wg][gq + 8][d]);
-          oacc[i][0] = a0 * oacc[i][0] + b0 * x.x;
-          oacc[i][1] = a0 * oacc[i][1] + b0 * x.y;
-          oacc[i][2] = a1 * oacc[i][2] + b1 * y.x;
-          oacc[i][3] = a1 * oacc[i][3] + b1 * y.y;
-        }
+      for (int i = 0; i < 16; ++i) {
+        const int d = i * 8 + 2 * cq;
+        const float2 x = *reinterpret_cast<const float2*>(&sm.ow[wg][gq][d]);
+        const float2 y = *reinterpret_cast<const float2*>(&sm.ow[wg][gq + 8][d]);
+        oacc[i][0] = a0 * oacc[i][0] + b0 * x.x;
+        oacc[i][1] = a0 * oacc[i][1] + b0 * x.y;
+        oacc[i][2] = a1 * oacc[i][2] + b1 * y.x;
+        oacc[i][3] = a1 * oacc[i][3] + b1 * y.y;
       }
-      __syncthreads();
-      // (2) group 0 publishes the folded states
-      if (grp == 0) {
-        if (cq == 0) {
-          sm.mw[wg][gq] = m0; sm.mw[wg][gq + 8] = m1;
-          sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
-        }
+    }
+    __syncthreads();
+    // (2) group 0 publishes the folded states
+    if (grp == 0) {
+      if (cq == 0) {
+        sm.mw[wg][gq] = m0; sm.mw[wg][gq + 8] = m1;
+        sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
+      }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int d = i * 8 + 2 * cq;
-          *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
-          *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
-        }
+      for (int i = 0; i < 16; ++i) {
+        const int d = i * 8 + 2 * cq;
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
+        *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
       }
-      __syncthreads();
-      const int64_t pbeg = sm.prefix[pc.pr], pend = sm.prefix[pc.pr + 1];
-      const int64_t c0 = (lo > pbeg ? lo : pbeg) - pbeg;
-      const int64_t c1 = (hi < pend ? hi : pend) - pbeg;
-      const bool whole = (c0 == 0) && (c1 == pend - pbeg);
+    }
+    __syncthreads();
+    {
       // 256 threads: thread t owns column d = t % 128 of rows r with r % 2 == t / 128
       const int d = tid % kDecD;
       const int rpar = tid / kDecD;
-      const int slot = (pc.pr == first_pair) ? 2 * cta : 2 * cta + 1;
+      const int slot = (pi == 0) ? 2 * cta : 2 * cta + 1;
       for (int rr = rpar; rr < p.rows; rr += 2) {
         float M = NEG;
         for (int w = 0; w < kDecGroupWarps; ++w) M = fmaxf(M, sm.mw[w][rr]);
@@ -612,13 +477,99 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
           if (d == 0) p.ws_lse[slot * kDecRows + rr] = lv;
         }
       }
-      if (!whole) finish_split(pc.pr);
-      __syncthreads();
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();  // the window's list and stages may be reused
+    __syncthreads();  // merge buffers free; this CTA's partial writes are issued
+    if (!whole && tid == 0) {
+      // Release this CTA's partial (the fence after the barrier covers the
+      // writes of every thread) and take a ticket; its value is read only
+      // after the whole range has been streamed.
+      __threadfence();
+      if (pi == 0) ticket0 = atomicAdd(p.ws_ticket + pr, 1);
+      else ticket1 = atomicAdd(p.ws_ticket + pr, 1);
+    }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  if (p.pair_mode) return;
 
+  // ---- shared pairs: the CTA that took the last ticket merges all partials
+  const int pr_first = static_cast<int>(lo / pp), pr_last = static_cast<int>((hi - 1) / pp);
+  const bool split0 = lo > static_cast<int64_t>(pr_first) * pp ||
+                      hi < static_cast<int64_t>(pr_first + 1) * pp;
+  const bool split1 = n_pieces > 1 && hi < static_cast<int64_t>(pr_last + 1) * pp;
+  auto ctas_sharing = [&](int pr) {
+    const int c_first = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid);
+    const int c_last = dec_cta_of(static_cast<int64_t>(pr + 1) * pp - 1, total, grid);
+    int n = 0;
+    for (int c = c_first; c <= c_last; ++c)
+      n += dec_range_lo(c, total, grid) < dec_range_lo(c + 1, total, grid) ? 1 : 0;
+    return n;
+  };
+  if (tid == 0) {
+    const int l0f = split0 && ticket0 == ctas_sharing(pr_first) - 1;
+    const int l1f = split1 && ticket1 == ctas_sharing(pr_last) - 1;
+    if (l0f || l1f) __threadfence();
+    sm.last[0] = l0f;
+    sm.last[1] = l1f;
+  }
+  __syncthreads();
+  for (int k = 0; k < 2; ++k) {
+    if (!sm.last[k]) continue;
+    const int pr = k == 0 ? pr_first : pr_last;
+    const int b = pr / p.Hkv, g = pr % p.Hkv;
+    const int c_first = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid);
+    const int c_last = dec_cta_of(static_cast<int64_t>(pr + 1) * pp - 1, total, grid);
+    const int d4 = (tid & 31) * 4;
+    // one warp per row, four columns per lane; partials fetched four CTAs at a time
+    for (int rr = warp; rr < p.rows; rr += kDecWarps) {
+      float M = NEG, W = 0.f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c0 = c_first; c0 <= c_last; c0 += 4) {
+        float lv[4];
+        float4 ov[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int cc = c0 + u;
+          lv[u] = NEG;
+          ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (cc <= c_last) {
+            const int64_t clo = dec_range_lo(cc, total, grid);
+            if (clo < dec_range_lo(cc + 1, total, grid)) {
+              const int sl = (clo / pp == pr) ? 2 * cc : 2 * cc + 1;
+              lv[u] = __ldcg(p.ws_lse + sl * kDecRows + rr);
+              ov[u] = __ldcg(reinterpret_cast<const float4*>(
+                  p.ws_part + (static_cast<int64_t>(sl) * kDecRows + rr) * kDecD + d4));
+            }
+          }
+        }
+        float Mn = M;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) Mn = fmaxf(Mn, lv[u]);
+        if (Mn == NEG) continue;
+        const float a = (M == NEG) ? 0.f : __expf(M - Mn);
+        W *= a;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] *= a;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float wt = (lv[u] == NEG) ? 0.f : __expf(lv[u] - Mn);
+          W += wt;
+          acc[0] += wt * ov[u].x;
+          acc[1] += wt * ov[u].y;
+          acc[2] += wt * ov[u].z;
+          acc[3] += wt * ov[u].w;
+        }
+        M = Mn;
+      }
+      const float inv = W > 0.f ? 1.f / W : 0.f;
+      const int sq = rr / p.G, h = g * p.G + rr % p.G;
+      __nv_bfloat16* op = p.o + b * p.osb + sq * p.oss + h * p.osh + d4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) op[e] = __float2bfloat16(acc[e] * inv);
+      if (lane == 0)
+        p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.Sq + sq] = W > 0.f ? M + __logf(W) : NEG;
+    }
+    if (tid == 0) p.ws_ticket[pr] = 0;
+  }
 }
 
 // ----------------------------------------------------------------------------

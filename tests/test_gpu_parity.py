@@ -158,6 +158,42 @@ def test_speculative_sparse_full_workload(sb):
     compare(o, lse, ro, rl, "spec decode full")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Lk,bs,spec,nmax", [
+    (1, 16, 1, 1, 8192, 256, 1000, 12),   # one pair spread over every CTA, 16 rows
+    (3, 4, 2, 2, 1000, 16, 100, 9),       # kv_block 16, ragged last block
+    (2, 8, 4, 1, 3000, 32, 1, 40),        # a one-key spec pass, many short blocks
+    (4, 4, 4, 4, 5000, 64, 777, 5),       # G = 1, Sq = 4
+])
+def test_speculative_sparse_edge_cases(sb, B, Hq, Hkv, Sq, Lk, bs, spec, nmax):
+    """Padding entries (-1) scattered through the table, one (b, kv-head) row
+    with only padding, a spec range that is not a multiple of 64 keys and a
+    key length that is not a multiple of the block size; the same workspace
+    is used twice in a row."""
+    rng = np.random.default_rng(B * 1000 + bs)
+    q = W.normal_bf16(rng, (B, Sq, Hq, 128))
+    k = W.normal_bf16(rng, (B, Lk, Hkv, 128))
+    v = W.normal_bf16(rng, (B, Lk, Hkv, 128))
+    ks, vs = k[:, Lk - spec:], v[:, Lk - spec:]
+    nkb = -(-Lk // bs)
+    tab = np.full((B, Hkv, 1, nmax), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            if b == B - 1 and g == 0:
+                continue                      # this row keeps only padding
+            sel = rng.choice(nkb, size=min(nmax, nkb), replace=False)
+            keep = rng.random(sel.size) < 0.8
+            tab[b, g, 0, :keep.sum()] = sel[keep]
+            rng.shuffle(tab[b, g, 0])
+    ws = sb.decode_workspace(B, Hkv, Sq, Hq, "cuda")
+    st = sb.new_status("cuda")
+    for _ in range(2):
+        o, lse = sb.speculative_sparse(dev(q), dev(ks), dev(vs), True, dev(k), dev(v),
+                                       torch.from_numpy(tab).cuda(), bs, ws=ws, status=st)
+    sb.check_status(st)
+    ro, rl = oracle.speculative_sparse(q, ks, vs, True, k, v, tab, bs, W.default_scale())
+    compare(o, lse, ro, rl, f"spec edge B={B} G={Hq // Hkv} Sq={Sq} bs={bs}")
+
+
 # ------------------------------------------------------------------ gated
 
 def _gated_small(L=1024, Hq=8, Hkv=2, k_top=4):
