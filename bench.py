@@ -257,20 +257,23 @@ def gated_flops(keep, L, Hq, block=64):
 
 
 def bench_gated(torch, sb, dist, args, flush, peaks):
-    T = np.load(os.path.join(ROOT, "tests", "golden", "gated_T_seed101.npy"))
-    wl = W.make_gated()
+    # T was calibrated at L = 32768; a shorter run (profiling) keeps its first
+    # L / 64 q-blocks, whose candidates j < i do not depend on L.
+    L = args.gated_len
+    T = np.load(os.path.join(ROOT, "tests", "golden", "gated_T_seed101.npy"))[:, :L // 64].copy()
+    wl = W.make_gated(L=L)
     q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
     Tg = torch.from_numpy(T).cuda()
     n = T.shape[1]
     keep = torch.zeros((1, 32, n, n), dtype=torch.uint8, device="cuda")
     o, lse = sb.fwd_gated(q, k, v, Tg, keep_out=keep)
     torch.cuda.synchronize()
-    flops, n_qk, n_pv = gated_flops(keep.cpu().numpy(), 32768, 32)
+    flops, n_qk, n_pv = gated_flops(keep.cpu().numpy(), L, 32)
     kept = int(keep.sum().item())
     ms, _ = time_device(torch, dist, lambda: sb.fwd_gated(q, k, v, Tg, out=o, lse=lse),
                         max(3, args.steps // 10), args.warmup, flush)
     tf = flops / (ms * 1e-3) / 1e12
-    return {"workload": "gated BSFA prefill B=1 Hq=32 Hkv=8 L=32768 causal D=128 bf16 64x64 "
+    return {"workload": f"gated BSFA prefill B=1 Hq=32 Hkv=8 L={L} causal D=128 bf16 64x64 "
                         "tiles, T from seed-101 calibration (k=64)",
             "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
             "kept_tile_density": round(kept / (32 * n * (n + 1) / 2), 4),
@@ -332,15 +335,16 @@ def nsa_pairs(wl):
 
 
 def bench_nsa(torch, sb, dist, args, flush, peaks):
-    wl = W.make_nsa_varlen()
+    seqlens = tuple(int(x) for x in args.nsa_seqlens.split(","))
+    wl = W.make_nsa_varlen(seqlens=seqlens)
     q, k, v = (W.to_torch_bf16(x, "cuda")[0] for x in (wl.q, wl.k, wl.v))
     cu = torch.from_numpy(wl.meta["cu_seqlens"]).cuda()
     sel = torch.from_numpy(wl.meta["sel"]).cuda()
     total, H = q.shape[0], q.shape[1]
-    ws = sb.varlen_selected_workspace(2, total, 65536, H, H, 16, "cuda")
+    ws = sb.varlen_selected_workspace(len(seqlens), total, max(seqlens), H, H, 16, "cuda")
     o = torch.empty_like(q)
     lse = torch.empty(H, total, dtype=torch.float32, device="cuda")
-    step = lambda: sb.fwd_varlen_selected(q, k, v, cu, 65536, sel, ws=ws, out=o, lse=lse)  # noqa: E731
+    step = lambda: sb.fwd_varlen_selected(q, k, v, cu, max(seqlens), sel, ws=ws, out=o, lse=lse)  # noqa: E731
     step()
     torch.cuda.synchronize()
     pairs = nsa_pairs(wl)
@@ -348,13 +352,14 @@ def bench_nsa(torch, sb, dist, args, flush, peaks):
     ms, _ = time_device(torch, dist, step, max(3, args.steps // 10), args.warmup, flush)
     tf = flops / (ms * 1e-3) / 1e12
     part_bytes = total * H * 16 * (128 + 1) * 4
-    return {"workload": "NSA selected attention, varlen cu_seqlens [0, 65536, 98304], Hq=Hkv=4, "
+    cu_txt = ", ".join(str(int(x)) for x in wl.meta["cu_seqlens"])
+    return {"workload": f"NSA selected attention, varlen cu_seqlens [{cu_txt}], Hq=Hkv=4, "
                         "D=128, bf16, top-16 blocks of 64 (block 0, 2 local, 13 random)",
             "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
             "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "partials_bytes": part_bytes,
             "note": "block-major: per-(token, head, slot) fp32 partials written and re-read "
-                    "by the combine; six launches per step (index build, main, combine)"}
+                    "by the combine; six kernels and a memset per step (index build, unit table, main, combine)"}
 
 
 def bench_table(torch, sb, dist, args, flush, peaks):
@@ -409,8 +414,19 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time the decode headline only (same as --prefill none)")
+    ap.add_argument("--prefill", default="gated,vertical_slash,nsa_varlen,block_table",
+                    help="comma-separated prefill workloads to time after the headline, or none")
+    ap.add_argument("--gated-len", type=int, default=32768,
+                    help="sequence length of the gated workload (a multiple of 64, <= 32768)")
+    ap.add_argument("--nsa-seqlens", default="65536,32768",
+                    help="sequence lengths of the NSA varlen workload")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()
+    if args.headline_only:
+        args.prefill = "none"
     args.warmup = max(args.warmup, 3)
     dist = Dist()
     peaks, peak_kind = load_peaks()
@@ -455,9 +471,10 @@ def main():
     clocks = ClockSampler(dist.local).start()
     dec = bench_decode(torch, sb, dist, args, flush, peaks)
     prefill = {}
-    if not args.headline_only:
-        for name, fn in (("gated", bench_gated), ("vertical_slash", bench_vs),
-                         ("nsa_varlen", bench_nsa), ("block_table", bench_table)):
+    wanted = [] if args.prefill == "none" else args.prefill.split(",")
+    for name, fn in (("gated", bench_gated), ("vertical_slash", bench_vs),
+                     ("nsa_varlen", bench_nsa), ("block_table", bench_table)):
+        if name in wanted:
             try:
                 prefill[name] = fn(torch, sb, dist, args, flush, peaks)
             except Exception as e:  # report, keep the headline
@@ -465,7 +482,7 @@ def main():
     ck = clocks.stop()
 
     cpu = None
-    if dist.rank == 0 and dist.world == 1:
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_decode(dec["wl"])
     value = dec["gbs"] * dist.world
     achieved = dec["bytes"] / (dec["ms"] * 1e-3) / 1e9

@@ -18,10 +18,10 @@
 // At the end of its part of a pair the CTA merges its warps' running
 // (m, l, O) and writes either the final row (the pair lies wholly inside its
 // range) or an fp32 partial.  A shared pair is finished by whichever CTA
-// takes the last ticket: tickets are taken right after each partial is
-// written but read only when the CTA has streamed its whole range, so no
-// warp waits on another CTA's progress; that CTA merges all partials with
-// the LSE combine and resets the ticket.
+// takes the last ticket; a CTA takes its tickets (at most two: its first and
+// last pair) only once it has streamed its whole range, so no warp stalls on
+// a fence mid-stream and no warp ever waits on another CTA; the CTA holding
+// the last ticket merges all partials with the LSE combine and resets it.
 #pragma once
 
 #include "sbfa_ptx.cuh"
@@ -40,6 +40,7 @@ constexpr int kDecMaxPairs = 4096;
 constexpr int kDecMaxEntries = 1024;
 constexpr int kDecRows = 16;
 constexpr int kDecD = 128;
+constexpr int kDecSharers = 8;  // sharers of a pair listed ahead of time
 
 struct DecodeParams {
   int B, Sq, Hq, Hkv, G, rows;
@@ -74,6 +75,11 @@ struct DecSmem {
   float lw[kDecGroupWarps][kDecRows];
   int2 meta[kDecWarps][kDecWarpStages];  // slice in each stage: {key0, nk | src << 7 | pr << 8}
   int last[2];                           // this CTA finishes shared pair 0 / 1
+  // CTAs sharing this CTA's first / last pair: their partial slots (-1 for
+  // an empty range) when there are at most kDecSharers of them, and count
+  int share_slot[2][kDecSharers];
+  int share_n[2];
+  int share_many[2];
 };
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decode shared memory exceeds 227 KB");
@@ -247,60 +253,88 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
+  // pair of piece pi
+  auto piece_pair = [&](int pi) {
+    return p.pair_mode ? cta + pi * grid : static_cast<int>(lo / pp) + pi;
+  };
+  // Rows r0 = gq and r1 = gq + 8 of the M = 16 tile (row = sq * G + head in group)
+  // and their causal limits in source A (bottom-right aligned).
+  const int r0 = gq, r1 = gq + 8;
+  const bool v0 = r0 < p.rows, v1 = r1 < p.rows;
+  const int lim0 = v0 ? r0 / p.G + (p.S_A - p.Sq) : -1;
+  const int lim1 = v1 ? r1 / p.G + (p.S_A - p.Sq) : -1;
+  // Q fragments (A operand, 16 rows x 128) of pair pr.  Loaded one piece
+  // ahead, while the previous piece merges, so no warp waits for them.
+  uint32_t qa[8][4];
+  auto load_q = [&](int pr) {
+    const int b = pr / p.Hkv, g = pr % p.Hkv;
+    const __nv_bfloat16* q0 =
+        v0 ? p.q + b * p.qsb + (r0 / p.G) * p.qss + (g * p.G + r0 % p.G) * p.qsh : nullptr;
+    const __nv_bfloat16* q1 =
+        v1 ? p.q + b * p.qsb + (r1 / p.G) * p.qss + (g * p.G + r1 % p.G) * p.qsh : nullptr;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int d = ks * 16 + 2 * cq;
+      qa[ks][0] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d)) : 0u;
+      qa[ks][1] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d)) : 0u;
+      qa[ks][2] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d + 8)) : 0u;
+      qa[ks][3] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d + 8)) : 0u;
+    }
+  };
+
+  load_q(piece_pair(0));
   load_meta(0);
 #pragma unroll
   for (int s = 0; s < kDecWarpStages; ++s) issue(s);
 
+  // While the first copies are in flight: which CTAs share this CTA's first
+  // and last pair, and the partial slot each of them writes (the 64-bit
+  // divisions stay off the end of the kernel).
+  const int pr_first = static_cast<int>(lo / pp), pr_last = static_cast<int>((hi - 1) / pp);
+  if (!p.pair_mode && warp == kDecWarps - 1 && lane < 2 * kDecSharers) {
+    const int k = lane / kDecSharers, s = lane % kDecSharers;
+    const int pr = k == 0 ? pr_first : pr_last;
+    const int c_first = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid);
+    const int c_last = dec_cta_of(static_cast<int64_t>(pr + 1) * pp - 1, total, grid);
+    const int cc = c_first + s;
+    int slot = -1;
+    if (cc <= c_last) {
+      const int64_t clo = dec_range_lo(cc, total, grid);
+      if (clo < dec_range_lo(cc + 1, total, grid)) slot = (clo / pp == pr) ? 2 * cc : 2 * cc + 1;
+    }
+    sm.share_slot[k][s] = slot;
+    const unsigned mask = __ballot_sync(0xffffu, slot >= 0);
+    if (s == 0) {
+      sm.share_n[k] = __popc(mask >> (k * kDecSharers) & 0xffu);
+      sm.share_many[k] = c_last - c_first + 1 > kDecSharers;
+    }
+  }
+
   // running state of the piece in progress
-  uint32_t qa[8][4];
   float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
   float oacc[16][4];
-  bool v0 = false, v1 = false;
-  int lim0 = -1, lim1 = -1;
-  int ticket0 = 0, ticket1 = 0;  // thread 0: tickets of the shared first / last pair
   int j = 0;
 
   for (int pi = 0; pi < n_pieces; ++pi) {
     int pr;
     int64_t nb, ne;
     bool whole;
+    pr = piece_pair(pi);
     if (p.pair_mode) {
-      pr = cta + pi * grid;
       nb = static_cast<int64_t>(pi) * pp;
       ne = nb + pp;
       whole = true;
     } else {
-      pr = static_cast<int>(lo / pp) + pi;
       const int64_t a = static_cast<int64_t>(pr) * pp, e = a + pp;
       nb = (a > lo ? a : lo) - lo;
       ne = (e < hi ? e : hi) - lo;
       whole = a >= lo && e <= hi;
     }
     const int b = pr / p.Hkv, g = pr % p.Hkv;
-    {
-      // Q fragments (A operand, 16 rows x 128) and per-row causal limits
-      const int r0 = gq, r1 = gq + 8;
-      v0 = r0 < p.rows;
-      v1 = r1 < p.rows;
-      lim0 = v0 ? r0 / p.G + (p.S_A - p.Sq) : -1;
-      lim1 = v1 ? r1 / p.G + (p.S_A - p.Sq) : -1;
-      const __nv_bfloat16* q0 =
-          v0 ? p.q + b * p.qsb + (r0 / p.G) * p.qss + (g * p.G + r0 % p.G) * p.qsh : nullptr;
-      const __nv_bfloat16* q1 =
-          v1 ? p.q + b * p.qsb + (r1 / p.G) * p.qss + (g * p.G + r1 % p.G) * p.qsh : nullptr;
+    m0 = m1 = NEG;
+    l0 = l1 = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const int d = ks * 16 + 2 * cq;
-        qa[ks][0] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d)) : 0u;
-        qa[ks][1] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d)) : 0u;
-        qa[ks][2] = q0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + d + 8)) : 0u;
-        qa[ks][3] = q1 ? __ldg(reinterpret_cast<const unsigned int*>(q1 + d + 8)) : 0u;
-      }
-      m0 = m1 = NEG;
-      l0 = l1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-    }
+    for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
     const int j_end = static_cast<int>((ne - grp + 1) / 2);  // chunks with grp + 2 j < ne
     for (; j < j_end; ++j) {
       asm volatile("cp.async.wait_group %0;" ::"n"(kDecWarpStages - 1) : "memory");
@@ -396,6 +430,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       issue(j + kDecWarpStages);
     }
 
+    if (pi + 1 < n_pieces) load_q(piece_pair(pi + 1));  // this piece's Q is dead
     // ---- merge the eight warps' states for this pair
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -478,25 +513,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
         }
       }
     }
-    __syncthreads();  // merge buffers free; this CTA's partial writes are issued
-    if (!whole && tid == 0) {
-      // Release this CTA's partial (the fence after the barrier covers the
-      // writes of every thread) and take a ticket; its value is read only
-      // after the whole range has been streamed.
-      __threadfence();
-      if (pi == 0) ticket0 = atomicAdd(p.ws_ticket + pr, 1);
-      else ticket1 = atomicAdd(p.ws_ticket + pr, 1);
-    }
+    __syncthreads();  // merge buffers free
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   if (p.pair_mode) return;
 
   // ---- shared pairs: the CTA that took the last ticket merges all partials
-  const int pr_first = static_cast<int>(lo / pp), pr_last = static_cast<int>((hi - 1) / pp);
   const bool split0 = lo > static_cast<int64_t>(pr_first) * pp ||
                       hi < static_cast<int64_t>(pr_first + 1) * pp;
   const bool split1 = n_pieces > 1 && hi < static_cast<int64_t>(pr_last + 1) * pp;
-  auto ctas_sharing = [&](int pr) {
+  auto ctas_sharing = [&](int k, int pr) {
+    if (!sm.share_many[k]) return sm.share_n[k];
     const int c_first = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid);
     const int c_last = dec_cta_of(static_cast<int64_t>(pr + 1) * pp - 1, total, grid);
     int n = 0;
@@ -505,19 +532,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     return n;
   };
   if (tid == 0) {
-    const int l0f = split0 && ticket0 == ctas_sharing(pr_first) - 1;
-    const int l1f = split1 && ticket1 == ctas_sharing(pr_last) - 1;
-    if (l0f || l1f) __threadfence();
-    sm.last[0] = l0f;
-    sm.last[1] = l1f;
+    // One ticket per shared pair.  The add releases this CTA's partials (the
+    // barrier before it orders every thread's writes ahead of it) and, for
+    // the last taker, acquires those of the other sharers.
+    const int ticket0 = split0 ? atom_add_acq_rel_gpu(p.ws_ticket + pr_first, 1) : 0;
+    const int ticket1 = split1 ? atom_add_acq_rel_gpu(p.ws_ticket + pr_last, 1) : 0;
+    sm.last[0] = split0 && ticket0 == ctas_sharing(0, pr_first) - 1;
+    sm.last[1] = split1 && ticket1 == ctas_sharing(1, pr_last) - 1;
   }
   __syncthreads();
   for (int k = 0; k < 2; ++k) {
     if (!sm.last[k]) continue;
     const int pr = k == 0 ? pr_first : pr_last;
     const int b = pr / p.Hkv, g = pr % p.Hkv;
-    const int c_first = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid);
-    const int c_last = dec_cta_of(static_cast<int64_t>(pr + 1) * pp - 1, total, grid);
+    const bool many = sm.share_many[k];
+    int c_first = 0, c_last = kDecSharers - 1;
+    if (many) {
+      c_first = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid);
+      c_last = dec_cta_of(static_cast<int64_t>(pr + 1) * pp - 1, total, grid);
+    }
     const int d4 = (tid & 31) * 4;
     // one warp per row, four columns per lane; partials fetched four CTAs at a time
     for (int rr = warp; rr < p.rows; rr += kDecWarps) {
@@ -531,14 +564,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
           const int cc = c0 + u;
           lv[u] = NEG;
           ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          int sl = -1;
           if (cc <= c_last) {
-            const int64_t clo = dec_range_lo(cc, total, grid);
-            if (clo < dec_range_lo(cc + 1, total, grid)) {
-              const int sl = (clo / pp == pr) ? 2 * cc : 2 * cc + 1;
-              lv[u] = __ldcg(p.ws_lse + sl * kDecRows + rr);
-              ov[u] = __ldcg(reinterpret_cast<const float4*>(
-                  p.ws_part + (static_cast<int64_t>(sl) * kDecRows + rr) * kDecD + d4));
+            if (!many) {
+              sl = sm.share_slot[k][cc - c_first];
+            } else {
+              const int64_t clo = dec_range_lo(cc, total, grid);
+              if (clo < dec_range_lo(cc + 1, total, grid)) sl = (clo / pp == pr) ? 2 * cc : 2 * cc + 1;
             }
+          }
+          if (sl >= 0) {
+            lv[u] = __ldcg(p.ws_lse + sl * kDecRows + rr);
+            ov[u] = __ldcg(reinterpret_cast<const float4*>(
+                p.ws_part + (static_cast<int64_t>(sl) * kDecRows + rr) * kDecD + d4));
           }
         }
         float Mn = M;

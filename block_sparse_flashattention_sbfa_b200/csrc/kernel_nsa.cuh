@@ -7,13 +7,18 @@
 //   1. nsa_count_kernel / nsa_scan_kernel / nsa_fill_kernel build the
 //      inverted index: for each (kv-head g, block) the list of (token, slot)
 //      pairs that selected it (counting sort).
-//   2. nsa_main_kernel: one unit = one key block and up to 128 query rows
-//      (entries x G query heads) that selected it.  Q rows are gathered with
-//      cp.async into a 128B-swizzled tile, K/V come by TMA, S = Q K^T and
-//      O = P V run on tcgen05 with fp32 accumulators in TMEM.  Each row's
-//      result over that one block is an fp32 partial (o, lse) stored at its
+//   2. nsa_units_kernel flattens the units: one unit = one key block and up
+//      to 128 query rows (entries x G query heads) that selected it; the
+//      table row of unit u holds its key rows, list entries and kv head.
+//   3. nsa_main_kernel: every CTA takes a contiguous range of units (units
+//      of one key block are adjacent, so neighbouring CTAs share K/V tiles
+//      in L2).  Q rows are gathered four at a time by TMA (tile::gather4
+//      over a (token x head) row map) into a 128B-swizzled tile, K/V come by
+//      TMA, S = Q K^T and O = P V run on tcgen05 with fp32 accumulators in
+//      TMEM.  Each row's result over
+//      that one block is an fp32 partial (o, lse) stored at its
 //      (token, head, slot).
-//   3. nsa_combine_kernel merges the top-k partials of every (token, head)
+//   4. nsa_combine_kernel merges the top-k partials of every (token, head)
 //      with the LSE combine.
 #pragma once
 
@@ -34,6 +39,9 @@ struct NsaParams {
   int* offset;         // [Hkv * NB + 1]
   int* unit_prefix;    // [Hkv * NB + 1]
   int* list;           // [entries]
+  int4* unit_a;        // [max units] {first key row, first list entry, entries, kv head}
+  int2* unit_b;        // [max units] {sequence start, sequence end}
+  int max_units;
   float* part_o;       // [total * Hq * topk, 128]
   float* part_lse;     // [total * Hq * topk]
   __nv_bfloat16* o;
@@ -51,26 +59,39 @@ __device__ __forceinline__ int nsa_seq_of(const int* cu, int nseq, int t) {
   return lo;
 }
 
-// Validate one selection entry; returns the global block id or -1.
-__device__ __forceinline__ int nsa_block_id(const NsaParams& p, int s, int j) {
+// Count and fill walk the selection in tiles of kNsaTokTile tokens: each
+// warp takes one (kv head, slot) column at a time with its lanes on
+// consecutive tokens, so that equal key blocks within a warp (block 0, the
+// local blocks) take one atomic between them (__match_any_sync).
+constexpr int kNsaTokTile = 64;
+constexpr int kNsaIdxThreads = 256;
+
+__device__ __forceinline__ int nsa_key(const NsaParams& p, int t, int s, int c, bool report_bad) {
+  const int j = __ldg(p.sel + static_cast<int64_t>(t) * p.Hkv * p.topk + c);
   if (j < 0) return -1;
   const int L = __ldg(p.cu + s + 1) - __ldg(p.cu + s);
   if (j >= (L + 63) / 64) {
-    report(p.status, kDevBadIndex);
+    if (report_bad) report(p.status, kDevBadIndex);
     return -1;
   }
-  return s * p.nbps + j;
+  return (c / p.topk) * p.nseq * p.nbps + s * p.nbps + j;
 }
 
-__global__ void nsa_count_kernel(NsaParams p) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(p.total) * p.Hkv * p.topk;
-  if (i >= n) return;
-  const int t = static_cast<int>(i / (p.Hkv * p.topk));
-  const int g = static_cast<int>((i / p.topk) % p.Hkv);
-  const int s = nsa_seq_of(p.cu, p.nseq, t);
-  const int gb = nsa_block_id(p, s, p.sel[i]);
-  if (gb >= 0) atomicAdd(&p.count[g * p.nseq * p.nbps + gb], 1);
+__global__ void __launch_bounds__(kNsaIdxThreads) nsa_count_kernel(NsaParams p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_tok = p.Hkv * p.topk;
+  const int ta = blockIdx.x * kNsaTokTile + lane, tb = ta + 32;
+  const int sa = ta < p.total ? nsa_seq_of(p.cu, p.nseq, ta) : 0;
+  const int sb = tb < p.total ? nsa_seq_of(p.cu, p.nseq, tb) : 0;
+  for (int c = warp; c < per_tok; c += kNsaIdxThreads / 32) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int t = hf ? tb : ta;
+      const int key = t < p.total ? nsa_key(p, t, hf ? sb : sa, c, true) : -1;
+      const unsigned m = __match_any_sync(0xffffffffu, key);
+      if (key >= 0 && lane == __ffs(m) - 1) atomicAdd(&p.count[key], __popc(m));
+    }
+  }
 }
 
 // Single CTA: exclusive prefix sums of counts and of units per (g, block).
@@ -114,21 +135,26 @@ __global__ void nsa_scan_kernel(NsaParams p) {
   }
 }
 
-__global__ void nsa_fill_kernel(NsaParams p) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(p.total) * p.Hkv * p.topk;
-  if (i >= n) return;
-  const int t = static_cast<int>(i / (p.Hkv * p.topk));
-  const int g = static_cast<int>((i / p.topk) % p.Hkv);
-  const int slot = static_cast<int>(i % p.topk);
-  const int s = nsa_seq_of(p.cu, p.nseq, t);
-  const int j = p.sel[i];
-  if (j < 0) return;
-  const int L = p.cu[s + 1] - p.cu[s];
-  if (j >= (L + 63) / 64) return;  // reported by the count pass
-  const int key = g * p.nseq * p.nbps + s * p.nbps + j;
-  const int pos = p.offset[key] + atomicAdd(&p.cursor[key], 1);
-  p.list[pos] = t * p.topk + slot;
+__global__ void __launch_bounds__(kNsaIdxThreads) nsa_fill_kernel(NsaParams p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_tok = p.Hkv * p.topk;
+  const int ta = blockIdx.x * kNsaTokTile + lane, tb = ta + 32;
+  const int sa = ta < p.total ? nsa_seq_of(p.cu, p.nseq, ta) : 0;
+  const int sb = tb < p.total ? nsa_seq_of(p.cu, p.nseq, tb) : 0;
+  for (int c = warp; c < per_tok; c += kNsaIdxThreads / 32) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int t = hf ? tb : ta;
+      const int key = t < p.total ? nsa_key(p, t, hf ? sb : sa, c, false) : -1;
+      const unsigned m = __match_any_sync(0xffffffffu, key);
+      const int leader = __ffs(m) - 1;
+      int base = 0;
+      if (key >= 0 && lane == leader) base = atomicAdd(&p.cursor[key], __popc(m));
+      base = __shfl_sync(0xffffffffu, base, leader);
+      if (key >= 0)
+        p.list[p.offset[key] + base + __popc(m & ((1u << lane) - 1u))] = t * p.topk + c % p.topk;
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -143,49 +169,66 @@ struct NsaSmem {
   alignas(1024) uint8_t p[2][kPTileBytes];
   uint32_t tmem_base;
   int abort_flag;
-  uint64_t kv_full[2], q_full[2], buf_empty[2];
+  uint64_t k_full[2], v_full[2], q_full[2];
   uint64_t s_full[2], p_full[2], o_full[2];
 };
 
 struct NsaUnit {
-  int g, s, j, e0, ne;  // kv head, sequence, local block, first list entry, entries
+  int key0, e0, ne, g;  // first key row (global), first list entry, entries, kv head
+  int base, end;        // the sequence's token range [base, end)
 };
 
-__device__ __forceinline__ NsaUnit nsa_unit(const NsaParams& p, int u) {
+// One thread per unit: locate its (kv head, block) by binary search over
+// the unit prefix sums and write its table row.
+__global__ void nsa_units_kernel(NsaParams p) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
   const int n = p.Hkv * p.nseq * p.nbps;
+  const int n_units = p.unit_prefix[n];
+  if (u >= n_units || u >= p.max_units) return;
   int lo = 0, hi = n;  // unit_prefix[lo] <= u < unit_prefix[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(p.unit_prefix + mid) <= u) lo = mid; else hi = mid;
+    if (p.unit_prefix[mid] <= u) lo = mid; else hi = mid;
   }
-  // skip (g, block) pairs with no unit (equal prefixes)
-  while (lo + 1 < n && __ldg(p.unit_prefix + lo + 1) <= u) ++lo;
-  NsaUnit r;
-  r.g = lo / (p.nseq * p.nbps);
+  while (lo + 1 < n && p.unit_prefix[lo + 1] <= u) ++lo;  // skip blocks with no unit
+  const int g = lo / (p.nseq * p.nbps);
   const int gb = lo % (p.nseq * p.nbps);
-  r.s = gb / p.nbps;
-  r.j = gb % p.nbps;
+  const int s = gb / p.nbps, j = gb % p.nbps;
   const int per_unit = 128 / p.G;
-  const int chunk = u - __ldg(p.unit_prefix + lo);
-  const int cnt = __ldg(p.offset + lo + 1) - __ldg(p.offset + lo);
-  r.e0 = __ldg(p.offset + lo) + chunk * per_unit;
-  r.ne = min(per_unit, cnt - chunk * per_unit);
+  const int chunk = u - p.unit_prefix[lo];
+  const int cnt = p.offset[lo + 1] - p.offset[lo];
+  const int base = p.cu[s];
+  p.unit_a[u] = make_int4(base + j * 64, p.offset[lo] + chunk * per_unit,
+                          min(per_unit, cnt - chunk * per_unit), g);
+  p.unit_b[u] = make_int2(base, p.cu[s + 1]);
+}
+
+__device__ __forceinline__ NsaUnit nsa_unit(const NsaParams& p, int u) {
+  const int4 a = __ldg(p.unit_a + u);
+  const int2 b = __ldg(p.unit_b + u);
+  NsaUnit r;
+  r.key0 = a.x; r.e0 = a.y; r.ne = a.z; r.g = a.w;
+  r.base = b.x; r.end = b.y;
   return r;
 }
 
 __global__ void __launch_bounds__(kNsaThreads, 1)
-    nsa_main_kernel(const __grid_constant__ CUtensorMap mapK,
+    nsa_main_kernel(const __grid_constant__ CUtensorMap mapQ,
+                    const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const NsaParams p) {
   extern __shared__ uint8_t smem_raw[];
   NsaSmem& sm = *reinterpret_cast<NsaSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_units = __ldg(p.unit_prefix + p.Hkv * p.nseq * p.nbps);
+  const int n_all = min(__ldg(p.unit_prefix + p.Hkv * p.nseq * p.nbps), p.max_units);
+  // this CTA's units: the contiguous range [u_lo, u_lo + n_mine)
+  const int u_lo = static_cast<int>(static_cast<int64_t>(n_all) * blockIdx.x / gridDim.x);
+  const int n_mine = static_cast<int>(static_cast<int64_t>(n_all) * (blockIdx.x + 1) / gridDim.x) - u_lo;
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.kv_full[b], 1);
-      mbar_init(&sm.q_full[b], 2);
-      mbar_init(&sm.buf_empty[b], 128);
+      mbar_init(&sm.k_full[b], 1);
+      mbar_init(&sm.v_full[b], 1);
+      mbar_init(&sm.q_full[b], 2);  // one expect-tx arrival per producer warp
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.p_full[b], 128);
       mbar_init(&sm.o_full[b], 1);
@@ -204,45 +247,81 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
   const WaitCtx wctx{&sm.abort_flag, p.status};
 
   if (warp == 0 || warp == 3) {
-    // ===================== producers: K/V by TMA, Q rows by cp.async =====================
-    const int half = warp == 0 ? 0 : 1;  // rows [64*half, 64*half + 64)
-    int n = 0;
+    // ===================== producers: Q rows by TMA gather4, K/V by TMA =====================
+    // Warp `half` fills rows [64 half, 64 half + 64) of the Q tile: lane l
+    // gathers rows 64 half + 4 (l % 16) + {0..3}, columns [64 (l / 16), +64).
+    // Rows past the unit's entries repeat its first row (their scores are
+    // masked and their outputs dropped).  Unit rows and list entries are
+    // loaded one and two units ahead.
+    const int half = warp == 0 ? 0 : 1;
+    auto load_codes = [&](const NsaUnit& un, int& c0, int& c1) {
+      // list entries of rows 64 half + lane and 64 half + 32 + lane
+      const int r0 = half * 64 + lane, r1 = r0 + 32;
+      c0 = (r0 / p.G < un.ne) ? __ldg(p.list + un.e0 + r0 / p.G) : -1;
+      c1 = (r1 / p.G < un.ne) ? __ldg(p.list + un.e0 + r1 / p.G) : -1;
+    };
+    NsaUnit cur{}, nxt{};
+    int c0 = -1, c1 = -1, n0 = -1, n1 = -1, first = 0, first_n = 0;
+    if (n_mine > 0) {
+      cur = nsa_unit(p, u_lo);
+      load_codes(cur, c0, c1);
+      first = __ldg(p.list + cur.e0);
+    }
+    if (n_mine > 1) nxt = nsa_unit(p, u_lo + 1);
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
+    // Buffers of unit n (index n & 1) were last used by unit n - 2: Q and K
+    // are free once QK(n - 2) has completed (s_full), V once PV(n - 2) has
+    // (o_full), which comes after QK(n - 1) and so after Q(n - 1) landed.
+    for (int n = 0; n < n_mine && ok; ++n) {
       const int b = n & 1;
-      if (lane == 0) ok = mbar_wait(&sm.buf_empty[b], ((n >> 1) & 1) ^ 1u, wctx);
+      const uint32_t pw = ((n >> 1) & 1) ^ 1u;
+      if (n + 1 < n_mine) {
+        load_codes(nxt, n0, n1);
+        first_n = __ldg(p.list + nxt.e0);
+      }
+      NsaUnit nn{};
+      if (n + 2 < n_mine) nn = nsa_unit(p, u_lo + n + 2);
+      if (lane == 0) ok = mbar_wait(&sm.s_full[b], pw, wctx);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      const NsaUnit un = nsa_unit(p, u);
+      if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[b], 64 * 128 * 2);
       if (half == 0 && lane == 0) {
-        const int key0 = __ldg(p.cu + un.s) + un.j * 64;
-        mbar_arrive_expect_tx(&sm.kv_full[b], 2 * kTileBytes);
-        tma_load_4d(sm.k[b], &mapK, &sm.kv_full[b], 0, un.g, key0, 0);
-        tma_load_4d(sm.k[b] + 8192, &mapK, &sm.kv_full[b], 64, un.g, key0, 0);
-        tma_load_4d(sm.v[b], &mapV, &sm.kv_full[b], 0, un.g, key0, 0);
-        tma_load_4d(sm.v[b] + 8192, &mapV, &sm.kv_full[b], 64, un.g, key0, 0);
+        mbar_arrive_expect_tx(&sm.k_full[b], kTileBytes);
+        tma_load_4d(sm.k[b], &mapK, &sm.k_full[b], 0, cur.g, cur.key0, 0);
+        tma_load_4d(sm.k[b] + 8192, &mapK, &sm.k_full[b], 64, cur.g, cur.key0, 0);
       }
-      const uint32_t d0 = smem_u32(sm.q[b]);
-      for (int e = lane; e < 64 * 16; e += 32) {
-        const int r = half * 64 + (e >> 4), ch = e & 15;
-        const uint32_t saddr = d0 + (ch >> 3) * 16384 + sw128_off(r, ch & 7);
-        const int ent = r / p.G;
-        if (ent < un.ne) {
-          const int code = __ldg(p.list + un.e0 + ent);
-          const int t = code / p.topk;
-          const int h = un.g * p.G + r % p.G;
-          const __nv_bfloat16* src = p.q + static_cast<int64_t>(t) * p.qss + h * p.qsh + ch * 8;
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(src)
-                       : "memory");
-        } else {
-          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(saddr), "r"(0)
-                       : "memory");
-        }
-      }
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.q_full[b]);
+      {
+        const int quad = lane & 15, colh = lane >> 4;
+        const int rl = 4 * quad;  // first of this lane's four rows within the warp's 64
+        int y[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rw = rl + i;
+          // the sending lane's value is fixed per call: fetch both, choose here
+          const int v0 = __shfl_sync(0xffffffffu, c0, rw & 31);
+          const int v1 = __shfl_sync(0xffffffffu, c1, rw & 31);
+          const int code = rw < 32 ? v0 : v1;
+          const int r = half * 64 + rw;
+          const int t = (code >= 0 ? code : first) / p.topk;
+          y[i] = t * p.Hq + cur.g * p.G + r % p.G;
+        }
+        tma_gather4_2d(sm.q[b] + colh * 16384 + (half * 64 + rl) * 128, &mapQ, &sm.q_full[b],
+                       colh * 64, y[0], y[1], y[2], y[3]);
+      }
+      if (half == 0) {
+        if (lane == 0) {
+          ok = mbar_wait(&sm.o_full[b], pw, wctx);
+          if (ok) {
+            mbar_arrive_expect_tx(&sm.v_full[b], kTileBytes);
+            tma_load_4d(sm.v[b], &mapV, &sm.v_full[b], 0, cur.g, cur.key0, 0);
+            tma_load_4d(sm.v[b] + 8192, &mapV, &sm.v_full[b], 64, cur.g, cur.key0, 0);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      cur = nxt; nxt = nn;
+      c0 = n0; c1 = n1; first = first_n;
     }
   } else if (warp == 1) {
     // ===================== MMA issuer =====================
@@ -259,7 +338,7 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       auto issue_qk = [&](int n) -> bool {
         const int b = n & 1;
         const uint32_t ph = (n >> 1) & 1;
-        if (!mbar_wait(&sm.q_full[b], ph, wctx) || !mbar_wait(&sm.kv_full[b], ph, wctx))
+        if (!mbar_wait(&sm.q_full[b], ph, wctx) || !mbar_wait(&sm.k_full[b], ph, wctx))
           return false;
         tc_fence_after();
         const uint64_t qd = qdesc0 + (b * kQTileBytes >> 4);
@@ -276,7 +355,8 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       auto issue_pv = [&](int n) -> bool {
         const int b = n & 1;
         const uint32_t ph = (n >> 1) & 1;
-        if (!mbar_wait(&sm.p_full[b], ph, wctx)) return false;
+        if (!mbar_wait(&sm.p_full[b], ph, wctx) || !mbar_wait(&sm.v_full[b], ph, wctx))
+          return false;
         tc_fence_after();
         const uint64_t pd = pdesc0 + (b * kPTileBytes >> 4);
         const uint64_t vd = vdesc0 + (b * kTileBytes >> 4);
@@ -287,8 +367,6 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         umma_commit(&sm.o_full[b]);
         return true;
       };
-      int n_mine = 0;
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) ++n_mine;
       if (n_mine > 0) ok = issue_qk(0);
       for (int n = 0; n < n_mine && ok; ++n) {
         if (n + 1 < n_mine) ok = issue_qk(n + 1);
@@ -306,22 +384,29 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     const int quarter = warp & 3;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * 256;
     const float NEG = -INFINITY;
-    int n = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++n) {
-      if ((n & 1) != b) continue;
+    // this warpgroup's units n = b, b + 2, ...: row codes one unit ahead
+    NsaUnit un_next{};
+    int code_next = -1;
+    if (b < n_mine) {
+      un_next = nsa_unit(p, u_lo + b);
+      code_next = r / p.G < un_next.ne ? __ldg(p.list + un_next.e0 + r / p.G) : -1;
+    }
+    for (int n = b; n < n_mine && ok; n += 2) {
       const uint32_t ph = (n >> 1) & 1;
-      const NsaUnit un = nsa_unit(p, u);
-      const int ent = r / p.G;
-      const bool valid = ent < un.ne;
+      const NsaUnit un = un_next;
+      const int code = code_next;
+      if (n + 2 < n_mine) {
+        un_next = nsa_unit(p, u_lo + n + 2);
+        code_next = r / p.G < un_next.ne ? __ldg(p.list + un_next.e0 + r / p.G) : -1;
+      }
+      const bool valid = code >= 0;
       int t = 0, slot = 0, tl = 0, L = 0;
       if (valid) {
-        const int code = __ldg(p.list + un.e0 + ent);
         t = code / p.topk;
         slot = code % p.topk;
-        const int base = __ldg(p.cu + un.s);
-        tl = t - base;
-        L = __ldg(p.cu + un.s + 1) - base;
+        tl = t - un.base;
+        L = un.end - un.base;
       }
       // tcgen05.ld is warp-collective: the warp agrees before leaving
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], ph, wctx))) { ok = false; break; }
@@ -332,7 +417,7 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       float mx = NEG;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const int key = un.j * 64 + c;
+        const int key = un.key0 - un.base + c;
         const bool vis = valid && key < L && (!p.causal || key <= tl);
         s[c] = vis ? s[c] * p.scale_log2 : NEG;
         mx = fmaxf(mx, s[c]);
@@ -373,8 +458,6 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         }
       }
       if (valid) p.part_lse[prow_idx] = l > 0.f ? (mu + lg2_approx(l)) * 0.69314718055994531f : NEG;
-      tc_fence_before();
-      mbar_arrive(&sm.buf_empty[b]);
     }
   }
   tc_fence_before();

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -78,6 +79,22 @@ sbfa_status encode_bshd(CUtensorMap* map, const sbfa_t4& t, int B, int S, int H,
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.ptr, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SBFA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SBFA_OK;
+}
+
+// 2-D map over `rows` rows of 128 bf16 (row stride `row_stride` elements),
+// box 64 columns x 1 row: the source of tile::gather4 row gathers.
+sbfa_status encode_rows2d(CUtensorMap* map, const void* ptr, int64_t rows, int64_t row_stride) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return fail(SBFA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride * 2)};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SBFA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return SBFA_OK;
@@ -344,7 +361,8 @@ sbfa_status check_table(const sbfa_table* t, const sbfa_shape* s, bool prefill) 
 // NSA selected attention workspace
 // ---------------------------------------------------------------------------
 struct NsaWs {
-  size_t count, cursor, offset, unit_prefix, list, part_lse, part_o, total;
+  size_t count, cursor, offset, unit_prefix, list, unit_a, unit_b, part_lse, part_o, total;
+  int64_t max_units;
 };
 
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -358,6 +376,11 @@ NsaWs nsa_ws_layout(int nseq, int total, int max_seqlen, int Hq, int Hkv, int to
   w.offset = off; off += al256((nb + 1) * 4);
   w.unit_prefix = off; off += al256((nb + 1) * 4);
   w.list = off; off += al256(static_cast<size_t>(total) * Hkv * topk * 4);
+  // units: at most entries / rows-per-unit, plus one partial unit per block
+  const int64_t per_unit = std::max<int64_t>(1, 128 / std::max(1, Hq / Hkv));
+  w.max_units = static_cast<int64_t>(total) * Hkv * topk / per_unit + static_cast<int64_t>(nb);
+  w.unit_a = off; off += al256(static_cast<size_t>(w.max_units) * 16);
+  w.unit_b = off; off += al256(static_cast<size_t>(w.max_units) * 8);
   w.part_lse = off; off += al256(static_cast<size_t>(total) * Hq * topk * 4);
   w.part_o = off; off += al256(static_cast<size_t>(total) * Hq * topk * 128 * 4);
   w.total = off;
@@ -721,6 +744,10 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   p.offset = reinterpret_cast<int*>(w + L.offset);
   p.unit_prefix = reinterpret_cast<int*>(w + L.unit_prefix);
   p.list = reinterpret_cast<int*>(w + L.list);
+  p.unit_a = reinterpret_cast<int4*>(w + L.unit_a);
+  p.unit_b = reinterpret_cast<int2*>(w + L.unit_b);
+  if (L.max_units >= (1ll << 31)) return fail(SBFA_ERR_UNSUPPORTED, "too many units");
+  p.max_units = static_cast<int>(L.max_units);
   p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.o = static_cast<__nv_bfloat16*>(o.ptr); p.oss = o.ss; p.osh = o.sh;
@@ -728,17 +755,22 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   p.status = status;
   const int64_t nb = static_cast<int64_t>(Hkv) * nseq * p.nbps;
   if (nb > (1 << 26)) return fail(SBFA_ERR_UNSUPPORTED, "too many key blocks");
-  CUtensorMap mk, mv;
+  // q rows (token, head) flattened: row t * Hq + h
+  if (Hq > 1 && q.ss != static_cast<int64_t>(Hq) * q.sh)
+    return fail(SBFA_ERR_UNSUPPORTED, "q: token stride must equal Hq * head stride");
+  CUtensorMap mq, mk, mv;
+  SBFA_TRY(encode_rows2d(&mq, q.ptr, static_cast<int64_t>(total) * Hq, Hq > 1 ? q.sh : q.ss));
   SBFA_TRY(encode_bshd(&mk, k, 1, total, Hkv, 64));
   SBFA_TRY(encode_bshd(&mv, v, 1, total, Hkv, 64));
   SBFA_CUDA(cudaMemsetAsync(p.count, 0, nb * 4, st));
-  const int64_t n_sel = static_cast<int64_t>(total) * Hkv * topk;
-  const unsigned g1 = static_cast<unsigned>((n_sel + 255) / 256);
-  sbfa::nsa_count_kernel<<<g1, 256, 0, st>>>(p);
+  const unsigned g1 = static_cast<unsigned>((total + sbfa::kNsaTokTile - 1) / sbfa::kNsaTokTile);
+  sbfa::nsa_count_kernel<<<g1, sbfa::kNsaIdxThreads, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
   sbfa::nsa_scan_kernel<<<1, 1024, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
-  sbfa::nsa_fill_kernel<<<g1, 256, 0, st>>>(p);
+  sbfa::nsa_fill_kernel<<<g1, sbfa::kNsaIdxThreads, 0, st>>>(p);
+  SBFA_CUDA(cudaGetLastError());
+  sbfa::nsa_units_kernel<<<static_cast<unsigned>((L.max_units + 255) / 256), 256, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
   const size_t smem = sizeof(sbfa::NsaSmem) + 1024;
   static bool attr_set[64] = {false};
@@ -749,7 +781,7 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr_set[dev] = true;
   }
-  sbfa::nsa_main_kernel<<<di.sms, sbfa::kNsaThreads, smem, st>>>(mk, mv, p);
+  sbfa::nsa_main_kernel<<<di.sms, sbfa::kNsaThreads, smem, st>>>(mq, mk, mv, p);
   SBFA_CUDA(cudaGetLastError());
   const int64_t rows = static_cast<int64_t>(total) * Hq;
   sbfa::nsa_combine_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);

@@ -246,12 +246,14 @@ sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
  * selected blocks sel[t, h/G, :] (sequence-local block indices, -1 =
  * padding, distinct), clipped to its sequence and, if causal, to keys <= tl.
  * cu_seqlens: int32 [nseq + 1] (device), 0 = cu[0] < ... < cu[nseq] = total;
- * max_seqlen >= every sequence length.  q: (1, total, Hq, 128) view, k and v:
- * (1, total, Hkv, 128) views (sb ignored); o like q; lse: fp32 [Hq, total].
- * sel: int32 [total, Hkv, topk] contiguous.  block must be 64; Hq/Hkv must
- * divide 128.  ws: device workspace of sbfa_varlen_selected_workspace_size()
- * bytes (contents need no initialisation).  Runs six launches on `stream`:
- * inverted-index count / scan / fill, the block-major tcgen05 kernel that
+ * max_seqlen >= every sequence length.  q: (1, total, Hq, 128) view whose
+ * token stride is Hq times its head stride (rows (token, head) are gathered
+ * by TMA from that flattened view), k and v: (1, total, Hkv, 128) views (sb
+ * ignored); o like q; lse: fp32 [Hq, total].  sel: int32 [total, Hkv, topk]
+ * contiguous.  block must be 64; Hq/Hkv must divide 128.  ws: device
+ * workspace of sbfa_varlen_selected_workspace_size() bytes (contents need
+ * no initialisation).  Runs on `stream`: a memset and the inverted-index
+ * count / scan / fill, the unit table, the block-major tcgen05 kernel that
  * writes one fp32 partial (o, lse) per (token, head, slot), and the LSE
  * combine of each row's partials.
  */
