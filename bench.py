@@ -55,9 +55,17 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def source_sha():
+# sources each profiled kernel is built from (its ncu counters go stale when any changes)
+KERNEL_SOURCES = {
+    "decode_kernel": ("kernel_decode.cuh", "sbfa_ptx.cuh"),
+    "prefill_kernel": ("kernel_prefill.cuh", "sbfa_ptx.cuh"),
+    "nsa_main_kernel": ("kernel_nsa.cuh", "kernel_prefill.cuh", "sbfa_ptx.cuh"),
+}
+
+
+def source_sha(kernel):
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(CSRC, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -70,7 +78,7 @@ def ncu_traffic(kernel):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
-    if not e or e.get("source_sha") != source_sha():
+    if not e or e.get("source_sha") != source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -125,17 +133,24 @@ class ClockSampler:
 
 
 class Dist:
-    def __init__(self):
+    """One process per GPU (RANK / WORLD_SIZE / LOCAL_RANK from the launcher).
+    The only collectives are the barrier around the timed region and the
+    max of the per-rank times: the replicas exchange no data."""
+
+    def __init__(self, backend="nccl", device="cuda"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend, self.device = backend, device
         self.pg = None
 
     def init(self, torch):
         if self.world > 1:
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"timeout": datetime.timedelta(seconds=120)}
+            if self.backend == "nccl":
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(self.backend, **kw)
             self.pg = dist
 
     def barrier(self, torch):
@@ -145,13 +160,20 @@ class Dist:
     def max(self, torch, x):
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
+
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def whole_job_rate(units_per_rank, max_ms, world):
+    """Weak scaling: every rank processes the same units; the job's rate is
+    all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / (max_ms * 1e-3)
 
 
 def time_device(torch, dist, fn, steps, warmup, flush):
@@ -484,7 +506,7 @@ def main():
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_decode(dec["wl"])
-    value = dec["gbs"] * dist.world
+    value = whole_job_rate(dec["bytes"], dec["ms"], dist.world) / 1e9
     achieved = dec["bytes"] / (dec["ms"] * 1e-3) / 1e9
     peak = peaks["hbm_gbs"]
     line = {
