@@ -167,6 +167,9 @@ struct NsaSmem {
   alignas(1024) uint8_t k[2][kTileBytes];
   alignas(1024) uint8_t v[2][kTileBytes];
   alignas(1024) uint8_t p[2][kPTileBytes];
+  // epilogue staging: each softmax warp turns its 32 rows x 32 fp32 columns
+  // around here so that every store instruction writes whole 128-byte rows
+  alignas(16) float stage[8][32][32];
   uint32_t tmem_base;
   int abort_flag;
   uint64_t k_full[2], v_full[2], q_full[2];
@@ -415,12 +418,22 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       tmem_ld32(lane_addr, s);
       tmem_ld32(lane_addr + 32, s + 32);
       float mx = NEG;
+      const int kb = un.key0 - un.base;  // first key of the block, sequence-local
+      if (__all_sync(0xffffffffu, valid && kb + 63 < L && (!p.causal || kb + 63 <= tl))) {
+        // every key of the block is visible to every row of this warp
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int key = un.key0 - un.base + c;
-        const bool vis = valid && key < L && (!p.causal || key <= tl);
-        s[c] = vis ? s[c] * p.scale_log2 : NEG;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 64; ++c) {
+          s[c] *= p.scale_log2;
+          mx = fmaxf(mx, s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int key = kb + c;
+          const bool vis = valid && key < L && (!p.causal || key <= tl);
+          s[c] = vis ? s[c] * p.scale_log2 : NEG;
+          mx = fmaxf(mx, s[c]);
+        }
       }
       const float mu = (mx == NEG) ? 0.f : mx;
       float l = 0.f;
@@ -445,17 +458,29 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       const int h = un.g * p.G + r % p.G;
       const int64_t prow_idx = (static_cast<int64_t>(t) * p.Hq + h) * p.topk + slot;
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      // 32 columns at a time: each lane parks its row in the warp's staging
+      // tile (16-byte pieces rotated by row to spread the banks), then lane
+      // group i / 8 of each store writes the 128 contiguous bytes of one row
+      float (*stg)[32] = sm.stage[warp - 4];
       float ob[32];
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(lane_addr + 128 + c * 32, ob);
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + prow_idx * 128 + c * 32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(ob[4 * i] * inv, ob[4 * i + 1] * inv, ob[4 * i + 2] * inv,
-                                 ob[4 * i + 3] * inv);
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(&stg[lane][4 * (i ^ (lane & 7))]) =
+              make_float4(ob[4 * i] * inv, ob[4 * i + 1] * inv, ob[4 * i + 2] * inv,
+                          ob[4 * i + 3] * inv);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), piece = lane & 7;
+          const long long dst_row = __shfl_sync(0xffffffffu, valid ? prow_idx : -1ll, rr);
+          const float4 x = *reinterpret_cast<const float4*>(&stg[rr][4 * (piece ^ (rr & 7))]);
+          if (dst_row >= 0)
+            *reinterpret_cast<float4*>(p.part_o + dst_row * 128 + c * 32 + 4 * piece) = x;
         }
+        __syncwarp();
       }
       if (valid) p.part_lse[prow_idx] = l > 0.f ? (mu + lg2_approx(l)) * 0.69314718055994531f : NEG;
     }

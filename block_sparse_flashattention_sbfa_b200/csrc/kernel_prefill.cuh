@@ -692,12 +692,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           // exact block max of each 64 x 64 sub-tile (BSFA Figure 2a)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float wm = rm[h];
-            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 16));
-            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 8));
-            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 4));
-            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 2));
-            wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, 1));
+            const float wm = warp_max_f32(rm[h]);
             if (lane == 0) sm.red[t][dbuf][quarter][h] = wm;
           }
           bool fail = !okw;
