@@ -42,6 +42,7 @@ struct NsaParams {
   int4* unit_a;        // [max units] {first key row, first list entry, entries, kv head}
   int2* unit_b;        // [max units] {sequence start, sequence end}
   int max_units;
+  int hist_tokens;     // tokens per CTA of the shared-memory histogram kernels
   float* part_o;       // [total * Hq * topk, 128]
   float* part_lse;     // [total * Hq * topk]
   __nv_bfloat16* o;
@@ -91,6 +92,63 @@ __global__ void __launch_bounds__(kNsaIdxThreads) nsa_count_kernel(NsaParams p) 
       const unsigned m = __match_any_sync(0xffffffffu, key);
       if (key >= 0 && lane == __ffs(m) - 1) atomicAdd(&p.count[key], __popc(m));
     }
+  }
+}
+
+// Shared-memory histogram variants, used when the (kv head, block) key space
+// fits in shared memory: every CTA takes a contiguous token range, counts
+// its entries per key in shared memory, and touches each global counter once
+// per key it saw.  With thousands of entries per key this removes the
+// global-atomic bottleneck of the per-entry kernels above.
+constexpr int kNsaHistThreads = 1024;
+constexpr int kNsaHistMaxKeys = 16384;  // fill keeps two int arrays: 128 KB
+
+__global__ void __launch_bounds__(kNsaHistThreads) nsa_count_hist_kernel(NsaParams p) {
+  extern __shared__ int hist[];
+  const int n_keys = p.Hkv * p.nseq * p.nbps;
+  const int per_tok = p.Hkv * p.topk;
+  for (int i = threadIdx.x; i < n_keys; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * p.hist_tokens * per_tok;
+  const int64_t e1 = min(static_cast<int64_t>(blockIdx.x + 1) * p.hist_tokens,
+                         static_cast<int64_t>(p.total)) * per_tok;
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const int t = static_cast<int>(e / per_tok), c = static_cast<int>(e % per_tok);
+    const int key = nsa_key(p, t, nsa_seq_of(p.cu, p.nseq, t), c, true);
+    if (key >= 0) atomicAdd(&hist[key], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_keys; i += blockDim.x)
+    if (hist[i]) atomicAdd(&p.count[i], hist[i]);
+}
+
+__global__ void __launch_bounds__(kNsaHistThreads) nsa_fill_hist_kernel(NsaParams p) {
+  extern __shared__ int smem_i[];
+  const int n_keys = p.Hkv * p.nseq * p.nbps;
+  int* cnt = smem_i;            // this CTA's entries per key, then its cursor per key
+  int* base = smem_i + n_keys;  // first list position of this CTA's run per key
+  const int per_tok = p.Hkv * p.topk;
+  for (int i = threadIdx.x; i < n_keys; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * p.hist_tokens * per_tok;
+  const int64_t e1 = min(static_cast<int64_t>(blockIdx.x + 1) * p.hist_tokens,
+                         static_cast<int64_t>(p.total)) * per_tok;
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const int t = static_cast<int>(e / per_tok), c = static_cast<int>(e % per_tok);
+    const int key = nsa_key(p, t, nsa_seq_of(p.cu, p.nseq, t), c, false);
+    if (key >= 0) atomicAdd(&cnt[key], 1);
+  }
+  __syncthreads();
+  // reserve one contiguous run per key for this CTA's entries
+  for (int i = threadIdx.x; i < n_keys; i += blockDim.x) {
+    base[i] = cnt[i] ? p.offset[i] + atomicAdd(&p.cursor[i], cnt[i]) : 0;
+    cnt[i] = 0;
+  }
+  __syncthreads();
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const int t = static_cast<int>(e / per_tok), c = static_cast<int>(e % per_tok);
+    const int key = nsa_key(p, t, nsa_seq_of(p.cu, p.nseq, t), c, false);
+    if (key >= 0) p.list[base[key] + atomicAdd(&cnt[key], 1)] = t * p.topk + c % p.topk;
   }
 }
 

@@ -763,12 +763,32 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   SBFA_TRY(encode_bshd(&mk, k, 1, total, Hkv, 64));
   SBFA_TRY(encode_bshd(&mv, v, 1, total, Hkv, 64));
   SBFA_CUDA(cudaMemsetAsync(p.count, 0, nb * 4, st));
+  // inverted index: shared-memory histograms when the key space fits, else
+  // one global atomic per (warp, key)
+  const bool hist = nb <= sbfa::kNsaHistMaxKeys;
   const unsigned g1 = static_cast<unsigned>((total + sbfa::kNsaTokTile - 1) / sbfa::kNsaTokTile);
-  sbfa::nsa_count_kernel<<<g1, sbfa::kNsaIdxThreads, 0, st>>>(p);
+  p.hist_tokens = (total + di.sms - 1) / di.sms;
+  const unsigned gh = static_cast<unsigned>((total + p.hist_tokens - 1) / p.hist_tokens);
+  const size_t hsm = static_cast<size_t>(nb) * 4;
+  static bool hist_attr[64] = {false};
+  int hdev = 0;
+  SBFA_CUDA(cudaGetDevice(&hdev));
+  if (hist && !hist_attr[hdev]) {
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::nsa_count_hist_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   sbfa::kNsaHistMaxKeys * 4));
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::nsa_fill_hist_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   sbfa::kNsaHistMaxKeys * 8));
+    hist_attr[hdev] = true;
+  }
+  if (hist) sbfa::nsa_count_hist_kernel<<<gh, sbfa::kNsaHistThreads, hsm, st>>>(p);
+  else sbfa::nsa_count_kernel<<<g1, sbfa::kNsaIdxThreads, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
   sbfa::nsa_scan_kernel<<<1, 1024, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
-  sbfa::nsa_fill_kernel<<<g1, sbfa::kNsaIdxThreads, 0, st>>>(p);
+  if (hist) sbfa::nsa_fill_hist_kernel<<<gh, sbfa::kNsaHistThreads, 2 * hsm, st>>>(p);
+  else sbfa::nsa_fill_kernel<<<g1, sbfa::kNsaIdxThreads, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
   sbfa::nsa_units_kernel<<<static_cast<unsigned>((L.max_units + 255) / 256), 256, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());

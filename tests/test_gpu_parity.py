@@ -327,6 +327,23 @@ def test_nsa_varlen_small_all_tokens(sb, seqlens):
     compare(o[None], lse[None], ro[None], rl[None], f"nsa small {seqlens}")
 
 
+def test_nsa_varlen_large_key_space(sb):
+    """max_seqlen far above the real lengths makes the (kv head, block) key
+    space too large for the shared-memory histograms: the inverted index is
+    built by the per-entry global-atomic kernels instead."""
+    seqlens = (600, 450)
+    wl = _nsa_case(seqlens, 2, 77)
+    cu, sel = wl.meta["cu_seqlens"], wl.meta["sel"]
+    q, k, v = (dev(x)[0] for x in (wl.q, wl.k, wl.v))
+    max_seqlen = 600000                      # 2 heads x 2 sequences x 9375 blocks
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_varlen_selected(q, k, v, torch.from_numpy(cu).cuda(), max_seqlen,
+                                    torch.from_numpy(sel).cuda(), status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_selected_varlen(wl.q[0], wl.k[0], wl.v[0], cu, sel, 64, True, wl.scale)
+    compare(o[None], lse[None], ro[None], rl[None], "nsa large key space")
+
+
 def test_nsa_varlen_full_workload_sampled(sb):
     """cu_seqlens [0, 65536, 98304], Hq=Hkv=4, top-16 blocks of 64; 4 whole
     64-token blocks (256 tokens) per head checked, incl. each sequence's last."""
