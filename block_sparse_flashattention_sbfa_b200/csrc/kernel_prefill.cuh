@@ -682,7 +682,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mask_half(sh, h);
             float m4[4] = {NEG, NEG, NEG, NEG};
 #pragma unroll
-            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sh[c]);
+            for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], sh[c], sh[c + 1]);
             rm[h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           }
         }
@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int c = 0; c < 4; ++c) {
             tmem_ld32(lane_addr + 128 + c * 32, ob);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ob[i] *= alpha;
+            for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], alpha);
             tmem_st32(lane_addr + 128 + c * 32, ob);
           }
         }
@@ -777,9 +777,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
-              const float p0 = ex2_approx(fmaf(sh[c], p.scale_log2, -base));
-              const float p1 = ex2_approx(fmaf(sh[c + 1], p.scale_log2, -base));
-              ps4[(c >> 1) & 3] += p0 + p1;
+              float x0, x1;
+              fma2(x0, x1, sh[c], sh[c + 1], p.scale_log2, -base);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              const int a = ((c >> 1) & 1) * 2;
+              add2(ps4[a], ps4[a + 1], p0, p1);
               pk[c >> 1] = pack_bf16x2(p0, p1);
             }
             psum += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
@@ -815,20 +817,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tmem_ld32(lane_addr + 128 + c * 32, ob);
           if (store) {
             const int64_t off = sc.b * p.osb + static_cast<int64_t>(my_row) * p.oss + head * p.osh + c * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], inv_l);
             if (p.o_f32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(ob[4 * i] * inv_l, ob[4 * i + 1] * inv_l,
-                                     ob[4 * i + 2] * inv_l, ob[4 * i + 3] * inv_l);
+                dst[i] = make_float4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
             } else {
               uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pack_bf16x2(ob[8 * i] * inv_l, ob[8 * i + 1] * inv_l),
-                                    pack_bf16x2(ob[8 * i + 2] * inv_l, ob[8 * i + 3] * inv_l),
-                                    pack_bf16x2(ob[8 * i + 4] * inv_l, ob[8 * i + 5] * inv_l),
-                                    pack_bf16x2(ob[8 * i + 6] * inv_l, ob[8 * i + 7] * inv_l));
+                dst[i] = make_uint4(pack_bf16x2(ob[8 * i], ob[8 * i + 1]),
+                                    pack_bf16x2(ob[8 * i + 2], ob[8 * i + 3]),
+                                    pack_bf16x2(ob[8 * i + 4], ob[8 * i + 5]),
+                                    pack_bf16x2(ob[8 * i + 6], ob[8 * i + 7]));
             }
           }
         }
