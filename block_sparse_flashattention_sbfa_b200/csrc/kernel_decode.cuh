@@ -443,10 +443,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
         sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 16; ++i) {  // rows past p.rows are never read back
         const int d = i * 8 + 2 * cq;
-        *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
-        *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
+        if (v0) *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
+        if (v1) *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
       }
     }
     __syncthreads();
@@ -463,8 +463,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int d = i * 8 + 2 * cq;
-        const float2 x = *reinterpret_cast<const float2*>(&sm.ow[wg][gq][d]);
-        const float2 y = *reinterpret_cast<const float2*>(&sm.ow[wg][gq + 8][d]);
+        const float2 x = v0 ? *reinterpret_cast<const float2*>(&sm.ow[wg][gq][d]) : make_float2(0.f, 0.f);
+        const float2 y = v1 ? *reinterpret_cast<const float2*>(&sm.ow[wg][gq + 8][d]) : make_float2(0.f, 0.f);
         oacc[i][0] = a0 * oacc[i][0] + b0 * x.x;
         oacc[i][1] = a0 * oacc[i][1] + b0 * x.y;
         oacc[i][2] = a1 * oacc[i][2] + b1 * y.x;
@@ -479,10 +479,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
         sm.lw[wg][gq] = l0; sm.lw[wg][gq + 8] = l1;
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 16; ++i) {  // rows past p.rows are never read back
         const int d = i * 8 + 2 * cq;
-        *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
-        *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
+        if (v0) *reinterpret_cast<float2*>(&sm.ow[wg][gq][d]) = make_float2(oacc[i][0], oacc[i][1]);
+        if (v1) *reinterpret_cast<float2*>(&sm.ow[wg][gq + 8][d]) = make_float2(oacc[i][2], oacc[i][3]);
       }
     }
     __syncthreads();

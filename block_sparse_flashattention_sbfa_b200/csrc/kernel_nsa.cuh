@@ -563,6 +563,48 @@ __global__ void nsa_combine_kernel(NsaParams p) {
   const int nb = (L + 63) / 64;
   const int* sl = p.sel + (static_cast<int64_t>(t) * p.Hkv + g) * p.topk;
   const int64_t row = (static_cast<int64_t>(t) * p.Hq + h) * p.topk;
+  if (p.topk <= 32) {
+    // lane k holds slot k's lse; the partial rows of the valid slots are
+    // then fetched eight at a time, all loads of a batch in flight together
+    float lv = -INFINITY;
+    if (lane < p.topk) {
+      const int j = __ldg(sl + lane);
+      if (j >= 0 && j < nb) lv = p.part_lse[row + lane];
+    }
+    const float M = warp_max_f32(lv);
+    const float Mn = (M == -INFINITY) ? 0.f : M;
+    const float w = (lv == -INFINITY) ? 0.f : __expf(lv - Mn);
+    float W = w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    unsigned vm = __ballot_sync(0xffffffffu, w > 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    while (vm) {
+      int ks[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        ks[u] = vm ? __ffs(vm) - 1 : -1;
+        vm &= vm - 1u;
+      }
+      float4 xs[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (ks[u] >= 0)
+          xs[u] = *reinterpret_cast<const float4*>(p.part_o + (row + ks[u]) * 128 + lane * 4);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (ks[u] < 0) continue;
+        const float wu = __shfl_sync(0xffffffffu, w, ks[u]);
+        acc.x += wu * xs[u].x; acc.y += wu * xs[u].y; acc.z += wu * xs[u].z; acc.w += wu * xs[u].w;
+      }
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    __nv_bfloat16* op = p.o + static_cast<int64_t>(t) * p.oss + h * p.osh + lane * 4;
+    reinterpret_cast<__nv_bfloat162*>(op)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    reinterpret_cast<__nv_bfloat162*>(op)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    if (lane == 0) p.lse[static_cast<int64_t>(h) * p.total + t] = W > 0.f ? Mn + __logf(W) : -INFINITY;
+    return;
+  }
   float M = -INFINITY;
   for (int k = 0; k < p.topk; ++k) {
     const int j = __ldg(sl + k);
