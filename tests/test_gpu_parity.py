@@ -308,6 +308,37 @@ def test_vertical_slash_columns_heavy(sb):
     compare(o, lse, ro, rl, "vs columns")
 
 
+def test_vertical_slash_full_workload_sampled(sb):
+    """L=131072, H=32, 1000 vertical columns and 6000 slash offsets per head,
+    64 x 64 blocks, causal.  The GPU's converted lists match the oracle's bit
+    for bit on every q-block of 8 heads, and on those heads 4 whole q-blocks
+    (256 rows, always including the last) match the oracle's attention."""
+    wl = W.make_vertical_slash()
+    L, H = wl.q.shape[1], wl.q.shape[2]
+    vert, slash = wl.meta["vertical"], wl.meta["slash"]
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    bc, bo, cc, ci = sb.convert_vertical_slash(sl, sl, torch.from_numpy(vert).cuda(),
+                                               torch.from_numpy(slash).cuda(), L)
+    o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), bc, bo, cc, ci, causal=True)
+    torch.cuda.synchronize()
+    heads = [0, 5, 11, 17, 22, 26, 29, 31]
+    hi = torch.tensor(heads, device="cuda")
+    gbc, gbo, gcc, gci = (x.index_select(1, hi).cpu().numpy() for x in (bc, bo, cc, ci))
+    del bo, ci
+    ref = [oracle.convert_vertical_slash([L], [L], vert[:, h:h + 1], slash[:, h:h + 1], L, 64,
+                                         64, True) for h in heads]
+    rbc, rbo, rcc, rci = (np.concatenate([r[i] for r in ref], axis=1) for i in range(4))
+    assert np.array_equal(gbc, rbc) and np.array_equal(gcc, rcc)
+    for idx in np.ndindex(rbc.shape):
+        assert np.array_equal(gbo[idx][:rbc[idx]], rbo[idx][:rbc[idx]])
+        assert np.array_equal(gci[idx][:rcc[idx]], rci[idx][:rcc[idx]])
+    rows = {j: sampled_rows(L, 64, 700 + h) for j, h in enumerate(heads)}
+    ro, rl = oracle.attend_vertical_slash(wl.q[:, :, heads], wl.k[:, :, heads], wl.v[:, :, heads],
+                                          rbc, rbo, rcc, rci, 64, 64, True, wl.scale,
+                                          rows=lambda b, j: rows[j])
+    compare(o[:, :, heads], lse[:, heads], ro, rl, "vs full")
+
+
 # ------------------------------------------------------------------ NSA selected (varlen)
 
 def _nsa_case(seqlens, H, seed):
