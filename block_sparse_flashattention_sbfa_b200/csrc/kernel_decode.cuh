@@ -231,6 +231,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
         const __nv_bfloat16* vrow0 =
             src ? p.vB + b * p.vBsb + g * p.vBsh : p.vA + b * p.vAsb + g * p.vAsh;
         const int64_t kro = src ? p.kBss : p.kAss, vro = src ? p.vBss : p.vAss;
+        // each K and V row is 256 contiguous bytes read by 16 lanes: the L2::256B
+        // qualifier lets the first copy bring in the whole row
         const uint32_t kdst = smem_u32(sm.slice[warp][stage]);
 #pragma unroll
         for (int it = 0; it < kDecSliceKeys * 16 / 32; ++it) {
@@ -240,10 +242,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
           const bool valid = kw + r < nk;
           const int64_t row = valid ? key0 + kw + r : 0;
           const uint32_t bytes = valid ? 16u : 0u;
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(kdst + off),
+          asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(kdst + off),
                        "l"(krow0 + row * kro + ch * 8), "r"(bytes)
                        : "memory");
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+          asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(
                            kdst + kDecSliceBytes / 2 + off),
                        "l"(vrow0 + row * vro + ch * 8), "r"(bytes)
                        : "memory");
