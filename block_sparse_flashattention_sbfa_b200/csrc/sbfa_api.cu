@@ -724,6 +724,9 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   SBFA_TRY(check_view(k, "k", true));
   SBFA_TRY(check_view(v, "v", true));
   SBFA_TRY(check_view(o, "o", false));
+  // q rows (token, head) are gathered from the flattened row t * Hq + h
+  if (Hq > 1 && q.ss != static_cast<int64_t>(Hq) * q.sh)
+    return fail(SBFA_ERR_UNSUPPORTED, "q: token stride must equal Hq * head stride");
   const NsaWs L = nsa_ws_layout(nseq, total, max_seqlen, Hq, Hkv, topk);
   if (ws_bytes < L.total)
     return fail(SBFA_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
@@ -755,9 +758,6 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   p.status = status;
   const int64_t nb = static_cast<int64_t>(Hkv) * nseq * p.nbps;
   if (nb > (1 << 26)) return fail(SBFA_ERR_UNSUPPORTED, "too many key blocks");
-  // q rows (token, head) flattened: row t * Hq + h
-  if (Hq > 1 && q.ss != static_cast<int64_t>(Hq) * q.sh)
-    return fail(SBFA_ERR_UNSUPPORTED, "q: token stride must equal Hq * head stride");
   CUtensorMap mq, mk, mv;
   SBFA_TRY(encode_rows2d(&mq, q.ptr, static_cast<int64_t>(total) * Hq, Hq > 1 ? q.sh : q.ss));
   SBFA_TRY(encode_bshd(&mk, k, 1, total, Hkv, 64));

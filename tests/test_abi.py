@@ -92,6 +92,17 @@ def test_host_validation_rejects_before_launch(sb):
                                            lse, lse, lse, None, None) == sb.ERR_UNSUPPORTED
     # combine: D must be 128
     assert lib.sbfa_combine(2, 1, 1, 1, 64, lse, lse, good, lse, None) == sb.ERR_UNSUPPORTED
+    # NSA varlen: q rows are gathered from the (token x head) flattening, so the
+    # token stride must be Hq head strides; and the selection block must be 64
+    ws = 1 << 20
+    q_bad = _t4(ss=4 * 128 + 64, sh=128)
+    assert lib.sbfa_fwd_varlen_selected(lse, 1, 8, 8, 4, 4, 128, 0.0, 1, q_bad, good, good, lse,
+                                        16, 64, ws, 1 << 30, good, lse, None, None) == \
+        sb.ERR_UNSUPPORTED
+    assert b"token stride" in lib.sbfa_last_error()
+    assert lib.sbfa_fwd_varlen_selected(lse, 1, 8, 8, 4, 4, 128, 0.0, 1, good, good, good, lse,
+                                        16, 32, ws, 1 << 30, good, lse, None, None) == \
+        sb.ERR_UNSUPPORTED
 
 
 def test_package_fails_loudly_without_library(tmp_path, monkeypatch):
