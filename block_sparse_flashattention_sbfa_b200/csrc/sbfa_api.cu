@@ -451,7 +451,11 @@ sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
   SBFA_TRY(check_view(k, "k", true));
   SBFA_TRY(check_view(v, "v", true));
   SBFA_TRY(check_outputs(o, lse));
-  const bool dec = decode_shape(shape) && table && table->q_block >= shape->Sq;
+  // short query blocks go to the split-KV kernel, which masks no table block:
+  // only when the call is not causal or has one query position (for which
+  // the bottom-right causal limit admits every key)
+  const bool dec = decode_shape(shape) && table && table->q_block >= shape->Sq &&
+                   (!shape->causal || shape->Sq == 1);
   SBFA_TRY(check_table(table, shape, !dec));
   if (dec) {
     sbfa::DecodeParams p{};

@@ -87,7 +87,8 @@ typedef struct {
  * of the blocks its table row lists (with the causal mask if shape->causal).
  * Constraints: kv_block in {64, 128, 256}; q_block a multiple of 64 (or
  * >= Sq); Sk <= 524288.  Decode shapes (Sq * Hq/Hkv <= 16 and one q-block)
- * run on the split-KV decode kernel, which also takes kv_block 16 and 32.
+ * that are not causal, or have Sq = 1, run on the split-KV decode kernel,
+ * which also takes kv_block 16 and 32.
  * Outputs: o (bf16, like q), lse (fp32 [B, Hq, Sq]).
  * status: optional device int32, SBFA_DEV_* bits are ORed in.
  */
