@@ -109,7 +109,10 @@ sbfa_status sbfa_fwd_dense(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t
  * Source: README, Usage 3 (per-block partials for a caller-side combine).
  * o_parts: fp32 [nmax, B, Sq, Hq, D] contiguous; lse_parts: fp32
  * [nmax, B, Hq, Sq] contiguous.  Partial n attends the keys of entry n of
- * each row's table (a padding entry gives o = 0, lse = -inf).
+ * each row's table (a padding entry gives o = 0, lse = -inf).  The combine
+ * of all nmax partials equals sbfa_fwd when a row lists each block once; a
+ * repeated entry yields a repeated partial, which the combine would count
+ * twice.
  */
 sbfa_status sbfa_fwd_partials(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
                               const sbfa_table* table, float* o_parts, float* lse_parts,
