@@ -199,16 +199,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
         src = 1;
         const int e = (c - nA) / cpe, sub = (c - nA) % cpe;
         const int b = pr / p.Hkv, g = pr % p.Hkv;
-        const int* row = p.idx + b * p.tsb + g * p.tsh;
-        const int jb = __ldg(row + e);
+        const int jb = __ldg(p.idx + b * p.tsb + g * p.tsh + e);
         if (jb >= 0 && jb < p.n_kb) {
-          // a block listed earlier in the row counts once: its repeat stays empty
-          bool dup = false;
-          for (int e2 = 0; e2 < e; ++e2) dup |= __ldg(row + e2) == jb;
-          if (!dup) {
-            key0 = jb * p.kv_block + sub * kDecChunk;
-            nk = max(min(kpc, p.S_B - key0), 0);
-          }
+          key0 = jb * p.kv_block + sub * kDecChunk;
+          nk = max(min(kpc, p.S_B - key0), 0);
         } else if (jb >= p.n_kb) {
           report(p.status, kDevBadIndex);
         }

@@ -71,8 +71,10 @@ typedef struct {
  * generalised per (batch, kv-head, q-block)).  Row r of query head h in
  * batch b uses idx[b*sb + (h/G)*sh + (r/q_block)*sqb + n], n < nmax.  Each
  * entry j >= 0 names the keys [j*kv_block, (j+1)*kv_block) clipped to Sk;
- * entries < 0 are padding; repeated entries count once; order does not
- * matter.  sb = sh = sqb = 0 broadcasts one 1-D table (the README's form).
+ * entries < 0 are padding; order does not matter.  A row must list each
+ * block at most once (a repeat is a precondition violation: the split-KV
+ * kernel would count it twice, the tiled kernel once).  sb = sh = sqb = 0
+ * broadcasts one 1-D table (the README's form).
  */
 typedef struct {
   const int32_t* idx;

