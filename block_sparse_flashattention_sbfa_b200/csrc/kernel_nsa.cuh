@@ -4,9 +4,13 @@
 // walking its own top-k blocks (one query row per kv-head: no tensor-core
 // tile), every selected key block gathers the query rows that chose it.
 //
-//   1. nsa_count_kernel / nsa_scan_kernel / nsa_fill_kernel build the
-//      inverted index: for each (kv-head g, block) the list of (token, slot)
-//      pairs that selected it (counting sort).
+//   1. count, scan and fill build the inverted index: for each (kv-head g,
+//      block) the list of (token, slot) pairs that selected it (a counting
+//      sort).  When the key space fits in shared memory each CTA histograms
+//      a token range there and touches each global counter once per key
+//      (nsa_count_hist_kernel / nsa_fill_hist_kernel); otherwise warps
+//      aggregate equal keys with __match_any_sync (nsa_count_kernel /
+//      nsa_fill_kernel).
 //   2. nsa_units_kernel flattens the units: one unit = one key block and up
 //      to 128 query rows (entries x G query heads) that selected it; the
 //      table row of unit u holds its key rows, list entries and kv head.
@@ -15,9 +19,9 @@
 //      in L2).  Q rows are gathered four at a time by TMA (tile::gather4
 //      over a (token x head) row map) into a 128B-swizzled tile, K/V come by
 //      TMA, S = Q K^T and O = P V run on tcgen05 with fp32 accumulators in
-//      TMEM.  Each row's result over
-//      that one block is an fp32 partial (o, lse) stored at its
-//      (token, head, slot).
+//      TMEM.  Each row's result over that one block is an fp32 partial
+//      (o, lse) stored at its (token, head, slot); the epilogue stages each
+//      warp's rows in shared memory so that stores write whole 128-byte rows.
 //   4. nsa_combine_kernel merges the top-k partials of every (token, head)
 //      with the LSE combine.
 #pragma once
