@@ -140,7 +140,11 @@ sbfa_status sbfa_combine(int32_t n_parts, int32_t B, int32_t Sq, int32_t Hq, int
  * over (a) all S_spec keys of (k_spec, v_spec), causal if causal_spec, and
  * (b) the blocks of (k, v) listed in `missed` (no mask), merged by the LSE
  * combine inside the kernel.  The result equals attention over the union.
- * shape->Sk is the length of k/v; shape->causal is ignored.
+ * shape->Sk is the length of k/v; shape->causal is ignored.  A paged KV
+ * cache is this call with k/v views of one page pool shared by all
+ * sequences (batch stride 0), kv_block = the page size, and each table row
+ * listing the pool pages of its missed blocks (FlagAttention's paged
+ * attention; pages may be shared between sequences).
  * Limits: Sq * (Hq/Hkv) <= 16; missed->q_block >= Sq; missed->kv_block in
  * {16, 32, 64, 128, 256}; B*Hkv <= 4096; missed->nmax <= 1024.
  * ws/ws_bytes: device workspace of at least sbfa_decode_workspace_size()

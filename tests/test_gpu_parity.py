@@ -222,6 +222,37 @@ def test_block_table_short_queries(sb, Sq, G, causal):
     compare(o, lse, ro, rl, f"short queries Sq={Sq} G={G} causal={causal}")
 
 
+def test_paged_kv_decode(sb):
+    """A paged KV cache through the same entry point: one physical pool of
+    pages shared by every sequence (k/v views with batch stride 0), each
+    (sequence, kv-head) row of the table listing the physical pages of its
+    missed blocks (kv_block = page size), pages shared between sequences
+    allowed.  Checked against attention over the union of the spec range
+    and the listed pages."""
+    rng = np.random.default_rng(91)
+    B, Hq, Hkv, page, n_pages, spec, nmax = 4, 16, 4, 128, 40, 300, 12
+    pool_k = W.normal_bf16(rng, (1, n_pages * page, Hkv, 128))
+    pool_v = W.normal_bf16(rng, (1, n_pages * page, Hkv, 128))
+    q = W.normal_bf16(rng, (B, 1, Hq, 128))
+    ks = W.normal_bf16(rng, (B, spec, Hkv, 128))
+    vs = W.normal_bf16(rng, (B, spec, Hkv, 128))
+    tab = np.stack([np.stack([rng.choice(n_pages, size=nmax, replace=False)
+                              for _ in range(Hkv)]) for _ in range(B)])[:, :, None, :]
+    tab = tab.astype(np.int32)
+    tab[3, 1, 0, 5:] = -1                      # a shorter page list
+    kd = dev(pool_k).expand(B, -1, -1, -1)     # batch stride 0: every sequence reads the pool
+    vd = dev(pool_v).expand(B, -1, -1, -1)
+    assert kd.stride(0) == 0
+    st = sb.new_status("cuda")
+    o, lse = sb.speculative_sparse(dev(q), dev(ks), dev(vs), True, kd, vd,
+                                   torch.from_numpy(tab).cuda(), page, status=st)
+    sb.check_status(st)
+    kl = np.broadcast_to(pool_k, (B,) + pool_k.shape[1:])
+    vl = np.broadcast_to(pool_v, (B,) + pool_v.shape[1:])
+    ro, rl = oracle.speculative_sparse(q, ks, vs, True, kl, vl, tab, page, W.default_scale())
+    compare(o, lse, ro, rl, "paged kv decode")
+
+
 # ------------------------------------------------------------------ gated
 
 def _gated_small(L=1024, Hq=8, Hkv=2, k_top=4):
