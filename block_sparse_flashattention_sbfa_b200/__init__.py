@@ -51,6 +51,7 @@ _SIGS = {
     "sbfa_fwd_partials": [ctypes.POINTER(Shape), T4, T4, T4, ctypes.POINTER(Table), _P, _P, _P,
                           _P],
     "sbfa_combine": [_I, _I, _I, _I, _I, _P, _P, T4, _P, _P],
+    "sbfa_calibrate_thresholds": [_P, _I, _I, _I, _I, _P, _P],
     "sbfa_speculative_sparse": [ctypes.POINTER(Shape), T4, T4, T4, _I, _I, T4, T4,
                                 ctypes.POINTER(Table), _P, ctypes.c_size_t, T4, _P, _P, _P],
     "sbfa_speculative_sparse_noalloc": [ctypes.POINTER(Shape), T4, T4, T4, _I, _I, T4, T4,
@@ -280,6 +281,22 @@ def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
           block_N, int(bool(causal)), bc.data_ptr(), bo.data_ptr(), cc.data_ptr(),
           ci.data_ptr(), _ptr(status), _stream())
     return bc, bo, cc, ci
+
+
+def calibrate_thresholds(smax, k_top, T=None):
+    """BSFA thresholds from block maxima (``sbfa_calibrate_thresholds``):
+    smax fp32 (B, Hq, n, n) -> T fp32 (B, Hq, n), T[b, h, i] = k-th largest
+    of smax[b, h, i, :i] (-inf when i < k)."""
+    if smax.dtype != torch.float32 or not smax.is_contiguous() or smax.dim() != 4:
+        raise TypeError("smax must be a contiguous fp32 (B, Hq, n, n) tensor")
+    B, Hq, n, n2 = smax.shape
+    if n != n2:
+        raise ValueError("smax must be square in its last two dims")
+    if T is None:
+        T = torch.empty(B, Hq, n, dtype=torch.float32, device=smax.device)
+    _call("sbfa_calibrate_thresholds", smax.data_ptr(), B, Hq, n, int(k_top), T.data_ptr(),
+          _stream())
+    return T
 
 
 def fwd_vertical_slash(q, k, v, block_count, block_offset, column_count, column_index,

@@ -119,4 +119,62 @@ __global__ void __launch_bounds__(kCvThreads)
   if (tid == 0) column_count[row] = ncol;
 }
 
+// ----------------------------------------------------------------------------
+// BSFA threshold calibration (Block Sparse Flash Attention, Figure 2a): for
+// every (batch, head, q-block i) T = the k-th largest of the off-diagonal
+// block maxima {s_max[i][j] : j < i}, counted with multiplicity, or -inf when
+// fewer than k candidates exist.  One CTA per row: exact radix selection over
+// the candidates' order-preserving 32-bit keys, eight bits per pass.
+// ----------------------------------------------------------------------------
+constexpr int kCalThreads = 256;
+
+__device__ __forceinline__ uint32_t cal_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(kCalThreads) calibrate_kernel(const float* __restrict__ smax,
+                                                                int n_qb, int k_top,
+                                                                float* __restrict__ T) {
+  __shared__ int hist[256];
+  __shared__ uint32_t sel_prefix;
+  __shared__ int sel_rank;
+  const int64_t row = blockIdx.x;             // (b * Hq + h) * n_qb + i
+  const int i = static_cast<int>(row % n_qb);
+  const float* cand = smax + row * n_qb;      // s_max[b][h][i][0..n_qb)
+  if (i < k_top) {                            // fewer than k candidates j < i
+    if (threadIdx.x == 0) T[row] = -INFINITY;
+    return;
+  }
+  uint32_t prefix = 0, mask = 0;
+  int rank = k_top;                           // 1-based rank from the top
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 256; b += kCalThreads) hist[b] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < i; j += kCalThreads) {
+      const uint32_t u = cal_key(cand[j]);
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int cum = 0, bucket = 0;
+      for (int b = 255; b >= 0; --b) {
+        if (cum + hist[b] >= rank) { bucket = b; break; }
+        cum += hist[b];
+      }
+      sel_prefix = prefix | (static_cast<uint32_t>(bucket) << shift);
+      sel_rank = rank - cum;
+    }
+    __syncthreads();
+    prefix = sel_prefix;
+    rank = sel_rank;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const uint32_t u = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
+    T[row] = __uint_as_float(u);
+  }
+}
+
 }  // namespace sbfa

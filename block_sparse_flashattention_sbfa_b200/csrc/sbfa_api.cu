@@ -813,6 +813,22 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   return SBFA_OK;
 }
 
+sbfa_status sbfa_calibrate_thresholds(const float* smax, int32_t B, int32_t Hq, int32_t n_qb,
+                                      int32_t k_top, float* T, sbfa_stream_t stream) {
+  g_last_error.clear();
+  if (!smax || !T) return fail(SBFA_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || Hq <= 0 || n_qb <= 0) return fail(SBFA_ERR_INVALID_ARG, "non-positive size");
+  if (k_top <= 0) return fail(SBFA_ERR_INVALID_ARG, "k must be positive");
+  const int64_t rows = static_cast<int64_t>(B) * Hq * n_qb;
+  if (rows >= (1ll << 31)) return fail(SBFA_ERR_UNSUPPORTED, "too many rows");
+  DevInfo di;
+  SBFA_TRY(dev_info(&di));
+  sbfa::calibrate_kernel<<<static_cast<unsigned>(rows), sbfa::kCalThreads, 0,
+                           reinterpret_cast<cudaStream_t>(stream)>>>(smax, n_qb, k_top, T);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
+}
+
 sbfa_status sbfa_check_status(const int32_t* status, sbfa_stream_t stream) {
   g_last_error.clear();
   SBFA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));

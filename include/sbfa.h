@@ -284,6 +284,19 @@ size_t sbfa_varlen_selected_workspace_size(int32_t nseq, int32_t total, int32_t 
  */
 sbfa_status sbfa_check_status(const int32_t* status, sbfa_stream_t stream);
 
+/*
+ * sbfa_calibrate_thresholds -- BSFA gate thresholds from block maxima.
+ * Source: Block Sparse Flash Attention, Figure 2a (calibration: the k-th
+ * largest off-diagonal block maximum of each row of blocks).  smax: fp32
+ * [B, Hq, n_qb, n_qb], as sbfa_fwd_gated writes to smax_out (only j < i is
+ * read; run the calibration pass with T = -inf to see every block).  T out:
+ * fp32 [B, Hq, n_qb] with T[b, h, i] = the k-th largest of
+ * {smax[b, h, i, j] : j < i}, counted with multiplicity, and -inf when
+ * i < k.  The selection is exact (no rounding).  One launch on `stream`.
+ */
+sbfa_status sbfa_calibrate_thresholds(const float* smax, int32_t B, int32_t Hq, int32_t n_qb,
+                                      int32_t k_top, float* T, sbfa_stream_t stream);
+
 /* Message of the last error on this host thread ("" if none). */
 const char* sbfa_last_error(void);
 

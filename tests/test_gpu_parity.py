@@ -324,6 +324,37 @@ def test_gated_full_workload_sampled(sb):
         compare(o, lse, ro, rl, "gated full")
 
 
+def test_calibrate_thresholds_exact(sb):
+    """GPU calibration (k-th largest off-diagonal block maximum per q-block)
+    on the block maxima the gated kernel writes, bit for bit against the
+    oracle's selection on the same values; ties counted with multiplicity on
+    a small-integer matrix; and within 1e-3 of thresholds built from the
+    oracle's own fp64 block maxima."""
+    cal = W.make_gated(B=1, Hq=8, Hkv=2, L=2048, seed=31)
+    n = 2048 // 64
+    smax = torch.empty((1, 8, n, n), device="cuda")
+    sb.fwd_gated(dev(cal.q), dev(cal.k), dev(cal.v),
+                 torch.full((8, n), -float("inf"), device="cuda"), smax_out=smax)
+    sm = smax.cpu().numpy()[0].astype(np.float64)
+    for k_top in (1, 4, 16, n):
+        Tg = sb.calibrate_thresholds(smax, k_top).cpu().numpy()[0].astype(np.float64)
+        assert np.array_equal(Tg, oracle.calibrate_thresholds(sm, k_top)), k_top
+    ties = torch.randint(-3, 4, (2, 3, 40, 40), device="cuda").float()
+    Tt = sb.calibrate_thresholds(ties.contiguous(), 5).cpu().numpy().astype(np.float64)
+    for b in range(2):
+        assert np.array_equal(Tt[b], oracle.calibrate_thresholds(ties[b].cpu().numpy().astype(np.float64), 5))
+    G = 4
+    ref = np.stack([oracle.block_max_head(cal.q[0, :, h], cal.k[0, :, h // G], 64, cal.scale)
+                    for h in range(8)])
+    Tr = oracle.calibrate_thresholds(ref, 4)
+    Tg = sb.calibrate_thresholds(smax, 4).cpu().numpy()[0].astype(np.float64)
+    fin = np.isfinite(Tr)
+    assert np.array_equal(fin, np.isfinite(Tg))
+    err = np.abs(Tg[fin] - Tr[fin]).max()
+    print(f"calibration: T max-abs vs fp64 block maxima {err:.2e}")
+    assert err < 1e-3
+
+
 # ------------------------------------------------------------------ vertical-slash
 
 def _vs_small(L=2048, H=4, nnz_v=64, nnz_s=160, seed=40):
