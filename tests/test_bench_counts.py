@@ -1,0 +1,98 @@
+"""The algorithmic work behind every number bench.py reports, checked
+against brute-force counts on small inputs (CPU).
+
+bench.py divides by these counts: kept K/V bytes for the decode GB/s, and
+exact visible (row, key) pairs for the prefill TFLOP/s.  Each count is
+recomputed here element by element from the same tables, masks and lists."""
+import importlib.util
+import os
+
+import numpy as np
+
+import oracle
+import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_decode_bytes_count_every_kept_key_once():
+    bm = _bench()
+    wl = W.make_spec_decode(B=2, Hq=8, Hkv=2, Lq=1, Lk=1000, block=128, spec_len=200,
+                            n_missed=3, seed=5, table_seed=6)
+    total, kv = bm.decode_bytes(wl)
+    t = wl.meta["table"]
+    keys = 0
+    for b in range(2):
+        for g in range(2):
+            seen = np.zeros(1000, dtype=bool)
+            for j in t[b, g, 0]:
+                if j >= 0:
+                    seen[j * 128:min((j + 1) * 128, 1000)] = True
+            keys += 200 + int(seen.sum())      # the spec range, then the listed blocks
+    assert kv == keys * 128 * 2 * 2             # K and V rows, bf16
+    assert total == kv + 2 * 2 * 1 * 8 * 128 * 2 + 2 * 8 * 1 * 4 + t.size * 4
+
+
+def test_gated_flops_match_pair_counts_of_the_keep_mask():
+    bm = _bench()
+    rng = np.random.default_rng(3)
+    L, H, blk = 640, 3, 64
+    n = L // blk
+    keep = np.zeros((1, H, n, n), dtype=np.uint8)
+    for h in range(H):
+        for i in range(n):
+            keep[0, h, i, :i + 1] = rng.random(i + 1) < 0.4
+            keep[0, h, i, i] = 1
+    flops, n_qk, n_pv = bm.gated_flops(keep, L, H)
+    r = np.arange(L)
+    causal = r[None, :] <= r[:, None]             # [row, key]
+    qk = H * int(causal.sum())
+    pv = 0
+    for h in range(H):
+        kept = np.kron(keep[0, h].astype(bool), np.ones((blk, blk), dtype=bool))
+        pv += int((kept & causal).sum())
+    assert (n_qk, n_pv) == (qk, pv)
+    assert flops == 2 * 128 * (qk + pv)
+
+
+def test_vertical_slash_flops_match_visible_pairs():
+    bm = _bench()
+    L, H = 1024, 2
+    vert, slash = W.vertical_slash_indices(np.random.default_rng(11), 1, H, L, 80, 120)
+    bc, bo, cc, ci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    flops, pairs = bm.vs_flops(bc, bo, cc, ci, L)
+    count = 0
+    r = np.arange(L)
+    for h in range(H):
+        for i in range(L // 64):
+            rows = r[i * 64:(i + 1) * 64]
+            keys = set()
+            for off in bo[0, h, i, :bc[0, h, i]]:
+                keys.update(range(off, min(off + 64, L)))
+            keys.update(int(c) for c in ci[0, h, i, :cc[0, h, i]])
+            kk = np.array(sorted(keys), dtype=np.int64)
+            count += int((kk[None, :] <= rows[:, None]).sum())
+    assert pairs == count
+    assert flops == 4 * 128 * count
+
+
+def test_nsa_pairs_match_visible_pairs():
+    bm = _bench()
+    wl = W.make_nsa_varlen(seqlens=(300, 130), H=2, seed=9, table_seed=19)
+    cu, sel = wl.meta["cu_seqlens"], wl.meta["sel"]
+    count = 0
+    for s in range(len(cu) - 1):
+        for t in range(cu[s], cu[s + 1]):
+            tl = t - cu[s]
+            for g in range(sel.shape[1]):
+                for j in sel[t, g]:
+                    if j >= 0:
+                        count += max(0, min(64, tl - 64 * int(j) + 1))
+    assert bm.nsa_pairs(wl) == count
