@@ -295,11 +295,17 @@ def bench_gated(torch, sb, dist, args, flush, peaks):
     ms, _ = time_device(torch, dist, lambda: sb.fwd_gated(q, k, v, Tg, out=o, lse=lse),
                         max(3, args.steps // 10), args.warmup, flush)
     tf = flops / (ms * 1e-3) / 1e12
-    return {"workload": f"gated BSFA prefill B=1 Hq=32 Hkv=8 L={L} causal D=128 bf16 64x64 "
-                        "tiles, T from seed-101 calibration (k=64)",
-            "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
-            "kept_tile_density": round(kept / (32 * n * (n + 1) / 2), 4),
-            "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+    res = {"workload": f"gated BSFA prefill B=1 Hq=32 Hkv=8 L={L} causal D=128 bf16 64x64 "
+                       "tiles, T from seed-101 calibration (k=64)",
+           "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
+           "kept_tile_density": round(kept / (32 * n * (n + 1) / 2), 4),
+           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+    if not args.no_cpu_baseline and dist.rank == 0:
+        try:
+            res["oracle"] = oracle_sample_gated(wl, T, flops)
+        except Exception as e:  # the GPU numbers stand without it
+            res["oracle"] = {"error": f"{type(e).__name__}: {e}"}
+    return res
 
 
 def vs_flops(bc, bo, cc, ci, L, block=64):
@@ -335,12 +341,18 @@ def bench_vs(torch, sb, dist, args, flush, peaks):
     cms, _ = time_device(torch, dist, conv, steps, 1, flush)
     tf = flops / (ms * 1e-3) / 1e12
     dense = 4 * 128 * 32 * L * (L + 1) // 2
-    return {"workload": "vertical-slash prefill B=1 H=32 L=131072 causal D=128 bf16 "
-                        "BM=BN=64, 1000 vertical + 6000 slash per head",
-            "ms": round(ms, 3), "tflops": round(tf, 2), "flops": flops,
-            "frac_of_causal_dense": round(flops / dense, 4),
-            "convert_ms": round(cms, 4),
-            "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+    res = {"workload": "vertical-slash prefill B=1 H=32 L=131072 causal D=128 bf16 "
+                       "BM=BN=64, 1000 vertical + 6000 slash per head",
+           "ms": round(ms, 3), "tflops": round(tf, 2), "flops": flops,
+           "frac_of_causal_dense": round(flops / dense, 4),
+           "convert_ms": round(cms, 4),
+           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+    if not args.no_cpu_baseline and dist.rank == 0:
+        try:
+            res["oracle"] = oracle_sample_vs(wl, flops)
+        except Exception as e:
+            res["oracle"] = {"error": f"{type(e).__name__}: {e}"}
+    return res
 
 
 def nsa_pairs(wl):
@@ -375,13 +387,19 @@ def bench_nsa(torch, sb, dist, args, flush, peaks):
     tf = flops / (ms * 1e-3) / 1e12
     part_bytes = total * H * 16 * (128 + 1) * 4
     cu_txt = ", ".join(str(int(x)) for x in wl.meta["cu_seqlens"])
-    return {"workload": f"NSA selected attention, varlen cu_seqlens [{cu_txt}], Hq=Hkv=4, "
+    res = {"workload": f"NSA selected attention, varlen cu_seqlens [{cu_txt}], Hq=Hkv=4, "
                         "D=128, bf16, top-16 blocks of 64 (block 0, 2 local, 13 random)",
             "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
             "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "partials_bytes": part_bytes,
             "note": "block-major: per-(token, head, slot) fp32 partials written and re-read "
                     "by the combine; six kernels and a memset per step (index build, unit table, main, combine)"}
+    if not args.no_cpu_baseline and dist.rank == 0:
+        try:
+            res["oracle"] = oracle_sample_nsa(wl, flops)
+        except Exception as e:
+            res["oracle"] = {"error": f"{type(e).__name__}: {e}"}
+    return res
 
 
 def bench_table(torch, sb, dist, args, flush, peaks):
@@ -424,6 +442,74 @@ def cpu_baseline_decode(wl, budget_s=15.0):
             "blas_threads": blas, "kind": "oracle",
             "sample": f"the whole decode workload (all 256 (b, h) rows), {done} pass(es), "
                       f"{sec:.2f} s per pass"}
+
+
+def _oracle_line(sec, sample_flops, full_flops, sample):
+    """The oracle's rate on a bounded sample and its time extrapolated to the
+    whole workload by the algorithmic FLOP count (pairs, not rows)."""
+    return {"value": round(sample_flops / sec / 1e12, 6), "unit": "TFLOP/s",
+            "cores": os.cpu_count(), "kind": "oracle", "sample": sample,
+            "sample_seconds": round(sec, 3),
+            "extrapolated_full_seconds": round(sec * full_flops / sample_flops, 1)}
+
+
+def oracle_sample_gated(wl, T, full_flops):
+    """Head 0, its last (heaviest) q-block: gate from fp64 block maxima, then
+    attention over the kept blocks."""
+    import oracle
+    L = wl.q.shape[1]
+    i = L // 64 - 1
+    rows = np.arange(i * 64, L)
+    t0 = time.perf_counter()
+    _, _, info = oracle.attend_gated(wl.q[:, :, :1], wl.k[:, :, :1], wl.v[:, :, :1], T[:1], 64,
+                                     wl.scale, rows=lambda b, h: rows, return_keep=True)
+    sec = time.perf_counter() - t0
+    keep = info[(0, 0, i)][1]
+    qk = int((rows + 1).sum())
+    pv = int(keep[:i].sum()) * 64 * 64 + 64 * 65 // 2
+    return _oracle_line(sec, 2 * 128 * (qk + pv), full_flops,
+                        f"head 0, q-block {i} (64 rows): gate over {i + 1} blocks, "
+                        f"{int(keep.sum())} kept")
+
+
+def oracle_sample_vs(wl, full_flops):
+    """Head 0: the oracle's conversion of its index lists, then attention for
+    its last (heaviest) q-block."""
+    import oracle
+    L = wl.q.shape[1]
+    vert, slash = wl.meta["vertical"][:, :1], wl.meta["slash"][:, :1]
+    i = L // 64 - 1
+    rows = np.arange(i * 64, L)
+    t0 = time.perf_counter()
+    bc, bo, cc, ci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    oracle.attend_vertical_slash(wl.q[:, :, :1], wl.k[:, :, :1], wl.v[:, :, :1], bc, bo, cc, ci,
+                                 64, 64, True, wl.scale, rows=lambda b, h: rows)
+    sec = time.perf_counter() - t0
+    offs = bo[0, 0, i, :bc[0, 0, i]] // 64
+    pairs = int((offs < i).sum()) * 64 * 64 + int((offs == i).sum()) * (64 * 65 // 2)
+    cols = ci[0, 0, i, :cc[0, 0, i]].astype(np.int64)
+    pairs += int(np.maximum(L - np.maximum(cols, i * 64), 0).sum())
+    return _oracle_line(sec, 4 * 128 * pairs, full_flops,
+                        f"head 0: index conversion for all {L // 64} q-blocks, attention for "
+                        f"q-block {i} (64 rows)")
+
+
+def oracle_sample_nsa(wl, full_flops, n_tok=256):
+    """Head 0, the last n_tok tokens of the first sequence (the most causal
+    keys)."""
+    import oracle
+    cu, sel = wl.meta["cu_seqlens"], wl.meta["sel"]
+    toks = np.arange(cu[1] - n_tok, cu[1])
+    t0 = time.perf_counter()
+    oracle.attend_selected_varlen(wl.q[0][:, :1], wl.k[0][:, :1], wl.v[0][:, :1], cu, sel[:, :1],
+                                  64, True, wl.scale, rows=lambda h: toks)
+    sec = time.perf_counter() - t0
+    tl = toks - cu[0]
+    s = sel[toks, 0].astype(np.int64)
+    cnt = np.clip(tl[:, None] - 64 * s + 1, 0, 64)
+    cnt[s < 0] = 0
+    return _oracle_line(sec, 4 * 128 * int(cnt.sum()), full_flops,
+                        f"head 0, the last {n_tok} tokens of sequence 0")
 
 
 # ----------------------------------------------------------------------------

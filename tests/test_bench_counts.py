@@ -96,3 +96,21 @@ def test_nsa_pairs_match_visible_pairs():
                     if j >= 0:
                         count += max(0, min(64, tl - 64 * int(j) + 1))
     assert bm.nsa_pairs(wl) == count
+
+
+def test_oracle_samples_beside_the_prefill_numbers():
+    """The bench's oracle-on-a-sample lines run on small workloads and report
+    a positive rate with a consistent extrapolation."""
+    bm = _bench()
+    wl = W.make_gated(B=1, Hq=4, Hkv=1, L=1024, seed=12)
+    sm = np.stack([oracle.block_max_head(wl.q[0, :, h], wl.k[0, :, 0], 64, wl.scale)
+                   for h in range(4)])
+    T = oracle.calibrate_thresholds(sm, 4).astype(np.float32)
+    g = bm.oracle_sample_gated(wl, T, full_flops=10 ** 12)
+    wv = W.make_vertical_slash(B=1, H=2, L=1024, nnz_v=80, nnz_s=120, seed=13, table_seed=14)
+    v = bm.oracle_sample_vs(wv, full_flops=10 ** 12)
+    wn = W.make_nsa_varlen(seqlens=(700, 300), H=2, seed=15, table_seed=16)
+    n = bm.oracle_sample_nsa(wn, full_flops=10 ** 12, n_tok=64)
+    for line in (g, v, n):
+        assert line["kind"] == "oracle" and line["value"] > 0 and line["sample_seconds"] > 0
+        assert line["extrapolated_full_seconds"] > line["sample_seconds"]
