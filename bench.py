@@ -58,7 +58,8 @@ def load_peaks():
 # sources each profiled kernel is built from (its ncu counters go stale when any changes)
 KERNEL_SOURCES = {
     "decode_kernel": ("kernel_decode.cuh", "sbfa_ptx.cuh"),
-    "prefill_kernel": ("kernel_prefill.cuh", "sbfa_ptx.cuh"),
+    "prefill_kernel<Gated>": ("kernel_prefill.cuh", "sbfa_ptx.cuh"),
+    "prefill_kernel<VS>": ("kernel_prefill.cuh", "sbfa_ptx.cuh"),
     "nsa_main_kernel": ("kernel_nsa.cuh", "kernel_prefill.cuh", "sbfa_ptx.cuh"),
 }
 
@@ -78,7 +79,7 @@ def ncu_traffic(kernel):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
-    if not e or e.get("source_sha") != source_sha(kernel):
+    if not e or kernel not in KERNEL_SOURCES or e.get("source_sha") != source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -170,6 +171,16 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def tensor_roofline(flops, ms, peaks, peak_kind, kernel, launches=1):
+    """Roofline object of a prefill step: algorithmic FLOPs over its CUDA-event
+    time, against the measured bf16 burst peak (the step is timed alone)."""
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "traffic": ncu_traffic(kernel), "peak_kind": peak_kind, "kernel": kernel,
+            "launches_per_step": launches, "algorithmic_flops": flops}
+
+
 def whole_job_rate(units_per_rank, max_ms, world):
     """Weak scaling: every rank processes the same units; the job's rate is
     all ranks' units over the slowest rank's time."""
@@ -177,7 +188,7 @@ def whole_job_rate(units_per_rank, max_ms, world):
 
 
 def time_device(torch, dist, fn, steps, warmup, flush):
-    """Per-step CUDA-event time of fn (ms, mean over steps; max over ranks).
+    """Per-step CUDA-event time of fn (ms, median over steps; max over ranks).
 
     The L2 flush runs before each step, outside the events; it is queued
     first so the GPU is still busy with it while the host issues the step,
@@ -198,7 +209,7 @@ def time_device(torch, dist, fn, steps, warmup, flush):
     torch.cuda.synchronize()
     dist.barrier(torch)
     wall = time.perf_counter() - t0
-    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
     return dist.max(torch, ms), wall
 
 
@@ -278,7 +289,7 @@ def gated_flops(keep, L, Hq, block=64):
     return 2 * 128 * n_qk + 2 * 128 * n_pv, n_qk, n_pv
 
 
-def bench_gated(torch, sb, dist, args, flush, peaks):
+def bench_gated(torch, sb, dist, args, flush, peaks, peak_kind):
     # T was calibrated at L = 32768; a shorter run (profiling) keeps its first
     # L / 64 q-blocks, whose candidates j < i do not depend on L.
     L = args.gated_len
@@ -299,7 +310,8 @@ def bench_gated(torch, sb, dist, args, flush, peaks):
                        "tiles, T from seed-101 calibration (k=64)",
            "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
            "kept_tile_density": round(kept / (32 * n * (n + 1) / 2), 4),
-           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+           "roofline": tensor_roofline(flops, ms, peaks, peak_kind, "prefill_kernel<Gated>")}
     if not args.no_cpu_baseline and dist.rank == 0:
         try:
             res["oracle"] = oracle_sample_gated(wl, T, flops)
@@ -322,7 +334,7 @@ def vs_flops(bc, bo, cc, ci, L, block=64):
     return 4 * 128 * pairs, pairs
 
 
-def bench_vs(torch, sb, dist, args, flush, peaks):
+def bench_vs(torch, sb, dist, args, flush, peaks, peak_kind):
     wl = W.make_vertical_slash()
     L = wl.q.shape[1]
     q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
@@ -346,10 +358,12 @@ def bench_vs(torch, sb, dist, args, flush, peaks):
            "ms": round(ms, 3), "tflops": round(tf, 2), "flops": flops,
            "frac_of_causal_dense": round(flops / dense, 4),
            "convert_ms": round(cms, 4),
-           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+           "roofline": tensor_roofline(flops, ms, peaks, peak_kind, "prefill_kernel<VS>")}
     if not args.no_cpu_baseline and dist.rank == 0:
         try:
             res["oracle"] = oracle_sample_vs(wl, flops)
+            res["oracle_convert"] = oracle_sample_vs_convert(wl)
         except Exception as e:
             res["oracle"] = {"error": f"{type(e).__name__}: {e}"}
     return res
@@ -368,7 +382,7 @@ def nsa_pairs(wl):
     return int(cnt.sum())
 
 
-def bench_nsa(torch, sb, dist, args, flush, peaks):
+def bench_nsa(torch, sb, dist, args, flush, peaks, peak_kind):
     seqlens = tuple(int(x) for x in args.nsa_seqlens.split(","))
     wl = W.make_nsa_varlen(seqlens=seqlens)
     q, k, v = (W.to_torch_bf16(x, "cuda")[0] for x in (wl.q, wl.k, wl.v))
@@ -391,6 +405,8 @@ def bench_nsa(torch, sb, dist, args, flush, peaks):
                         "D=128, bf16, top-16 blocks of 64 (block 0, 2 local, 13 random)",
             "ms": round(ms, 4), "tflops": round(tf, 2), "flops": flops,
             "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+            "roofline": tensor_roofline(flops, ms, peaks, peak_kind, "nsa_main_kernel",
+                                        launches=7),
             "partials_bytes": part_bytes,
             "note": "block-major: per-(token, head, slot) fp32 partials written and re-read "
                     "by the combine; six kernels and a memset per step (index build, unit table, main, combine)"}
@@ -402,7 +418,7 @@ def bench_nsa(torch, sb, dist, args, flush, peaks):
     return res
 
 
-def bench_table(torch, sb, dist, args, flush, peaks):
+def bench_table(torch, sb, dist, args, flush, peaks, peak_kind):
     wl = W.make_block_table()
     q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
     t = torch.from_numpy(wl.meta["table"]).cuda()
@@ -419,29 +435,36 @@ def bench_table(torch, sb, dist, args, flush, peaks):
 # CPU baseline: the oracle on the host cores
 # ----------------------------------------------------------------------------
 
-def cpu_baseline_decode(wl, budget_s=15.0):
+def cpu_baseline_decode(wl, steps=5, warmup=1):
+    """The oracle over the whole decode workload (every (b, h) row): `warmup`
+    untimed passes (they touch the inputs and warm the BLAS pools), then the
+    median of `steps` timed passes."""
     import oracle
     t = wl.meta["table"]
     s0 = wl.meta["spec_begin"]
     nbytes, _ = decode_bytes(wl)
-    t0 = time.perf_counter()
-    done = 0
-    while True:
+
+    def one():
         oracle.speculative_sparse(wl.q, wl.k[:, s0:], wl.v[:, s0:], True, wl.k, wl.v, t, 128,
                                   wl.scale)
-        done += 1
-        if time.perf_counter() - t0 > budget_s or done >= 3:
-            break
-    sec = (time.perf_counter() - t0) / done
+
+    for _ in range(warmup):
+        one()
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        one()
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
     try:
         from threadpoolctl import threadpool_info
         blas = max((x.get("num_threads", 1) for x in threadpool_info()), default=1)
     except Exception:
         blas = None
     return {"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": os.cpu_count(),
-            "blas_threads": blas, "kind": "oracle",
-            "sample": f"the whole decode workload (all 256 (b, h) rows), {done} pass(es), "
-                      f"{sec:.2f} s per pass"}
+            "blas_threads": blas, "kind": "oracle", "steps": steps, "warmup": warmup,
+            "sample": f"the whole decode workload (all 256 (b, h) rows) per pass; {warmup} "
+                      f"untimed pass(es), median of {steps} timed passes, {sec:.2f} s per pass"}
 
 
 def _oracle_line(sec, sample_flops, full_flops, sample):
@@ -449,8 +472,17 @@ def _oracle_line(sec, sample_flops, full_flops, sample):
     whole workload by the algorithmic FLOP count (pairs, not rows)."""
     return {"value": round(sample_flops / sec / 1e12, 6), "unit": "TFLOP/s",
             "cores": os.cpu_count(), "kind": "oracle", "sample": sample,
-            "sample_seconds": round(sec, 3),
+            "sample_seconds": round(sec, 3), "sample_flops": sample_flops,
             "extrapolated_full_seconds": round(sec * full_flops / sample_flops, 1)}
+
+
+def gated_sample_flops(i, keep, block=64):
+    """Algorithmic FLOPs of q-block i of one head (whole 64-row block): QK over
+    every causal key, PV over the kept off-diagonal blocks plus the diagonal."""
+    rows = np.arange(i * block, (i + 1) * block)
+    qk = int((rows + 1).sum())
+    pv = int(np.asarray(keep[:i]).sum()) * block * block + block * (block + 1) // 2
+    return 2 * 128 * (qk + pv)
 
 
 def oracle_sample_gated(wl, T, full_flops):
@@ -465,33 +497,65 @@ def oracle_sample_gated(wl, T, full_flops):
                                      wl.scale, rows=lambda b, h: rows, return_keep=True)
     sec = time.perf_counter() - t0
     keep = info[(0, 0, i)][1]
-    qk = int((rows + 1).sum())
-    pv = int(keep[:i].sum()) * 64 * 64 + 64 * 65 // 2
-    return _oracle_line(sec, 2 * 128 * (qk + pv), full_flops,
+    return _oracle_line(sec, gated_sample_flops(i, keep), full_flops,
                         f"head 0, q-block {i} (64 rows): gate over {i + 1} blocks, "
                         f"{int(keep.sum())} kept")
 
 
+def vs_sample_pairs(bc, bo, cc, ci, i, L, block=64):
+    """Visible (row, key) pairs of q-block i of head 0 under converted lists."""
+    offs = bo[0, 0, i, :bc[0, 0, i]] // block
+    pairs = int((offs < i).sum()) * block * block + int((offs == i).sum()) * (block * (block + 1) // 2)
+    cols = ci[0, 0, i, :cc[0, 0, i]].astype(np.int64)
+    m0, m1 = i * block, min((i + 1) * block, L)
+    pairs += int(np.minimum(block, np.maximum(m1 - np.maximum(cols, m0), 0)).sum())
+    return pairs
+
+
 def oracle_sample_vs(wl, full_flops):
-    """Head 0: the oracle's conversion of its index lists, then attention for
-    its last (heaviest) q-block."""
+    """Head 0, its last (heaviest) q-block: the oracle's attention over the
+    converted lists (the conversion of that q-block is done first and not
+    timed; oracle_sample_vs_convert times conversion on its own)."""
     import oracle
     L = wl.q.shape[1]
     vert, slash = wl.meta["vertical"][:, :1], wl.meta["slash"][:, :1]
     i = L // 64 - 1
     rows = np.arange(i * 64, L)
+    bc, bo, cc, ci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True,
+                                                   qblocks=[i])
     t0 = time.perf_counter()
-    bc, bo, cc, ci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
     oracle.attend_vertical_slash(wl.q[:, :, :1], wl.k[:, :, :1], wl.v[:, :, :1], bc, bo, cc, ci,
                                  64, 64, True, wl.scale, rows=lambda b, h: rows)
     sec = time.perf_counter() - t0
-    offs = bo[0, 0, i, :bc[0, 0, i]] // 64
-    pairs = int((offs < i).sum()) * 64 * 64 + int((offs == i).sum()) * (64 * 65 // 2)
-    cols = ci[0, 0, i, :cc[0, 0, i]].astype(np.int64)
-    pairs += int(np.maximum(L - np.maximum(cols, i * 64), 0).sum())
+    pairs = vs_sample_pairs(bc, bo, cc, ci, i, L)
     return _oracle_line(sec, 4 * 128 * pairs, full_flops,
-                        f"head 0: index conversion for all {L // 64} q-blocks, attention for "
-                        f"q-block {i} (64 rows)")
+                        f"head 0, q-block {i} (64 rows): attention over its converted lists")
+
+
+def oracle_sample_vs_convert(wl, n_qb=32):
+    """The oracle's index conversion on n_qb q-blocks of head 0 (the last
+    ones, whose causal range is the longest), extrapolated to every q-block of
+    every head; compare with the GPU's convert_ms."""
+    import oracle
+    L, H = wl.q.shape[1], wl.q.shape[2]
+    vert, slash = wl.meta["vertical"][:, :1], wl.meta["slash"][:, :1]
+    nqb = L // 64
+    qbs = list(range(nqb - n_qb, nqb))
+    t0 = time.perf_counter()
+    oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True, qblocks=qbs)
+    sec = time.perf_counter() - t0
+    return {"kind": "oracle", "unit": "s", "cores": os.cpu_count(),
+            "sample": f"conversion of {n_qb} q-blocks of head 0", "sample_seconds": round(sec, 3),
+            "extrapolated_full_seconds": round(sec * nqb * H / n_qb, 3)}
+
+
+def nsa_sample_pairs(cu, sel, toks):
+    """Visible (token, key) pairs of head 0 for tokens of sequence 0."""
+    tl = toks - cu[0]
+    s = sel[toks, 0].astype(np.int64)
+    cnt = np.clip(tl[:, None] - 64 * s + 1, 0, 64)
+    cnt[s < 0] = 0
+    return int(cnt.sum())
 
 
 def oracle_sample_nsa(wl, full_flops, n_tok=256):
@@ -504,11 +568,7 @@ def oracle_sample_nsa(wl, full_flops, n_tok=256):
     oracle.attend_selected_varlen(wl.q[0][:, :1], wl.k[0][:, :1], wl.v[0][:, :1], cu, sel[:, :1],
                                   64, True, wl.scale, rows=lambda h: toks)
     sec = time.perf_counter() - t0
-    tl = toks - cu[0]
-    s = sel[toks, 0].astype(np.int64)
-    cnt = np.clip(tl[:, None] - 64 * s + 1, 0, 64)
-    cnt[s < 0] = 0
-    return _oracle_line(sec, 4 * 128 * int(cnt.sum()), full_flops,
+    return _oracle_line(sec, 4 * 128 * nsa_sample_pairs(cu, sel, toks), full_flops,
                         f"head 0, the last {n_tok} tokens of sequence 0")
 
 
@@ -543,7 +603,7 @@ def main():
         if dist.rank != 0:
             return
         wl = W.make_spec_decode()
-        cb = cpu_baseline_decode(wl, budget_s=20.0)
+        cb = cpu_baseline_decode(wl, steps=args.steps, warmup=args.warmup)
         sec_per_step = decode_bytes(wl)[0] / (cb["value"] * 1e9)
         line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -584,14 +644,14 @@ def main():
                      ("nsa_varlen", bench_nsa), ("block_table", bench_table)):
         if name in wanted:
             try:
-                prefill[name] = fn(torch, sb, dist, args, flush, peaks)
+                prefill[name] = fn(torch, sb, dist, args, flush, peaks, peak_kind)
             except Exception as e:  # report, keep the headline
                 prefill[name] = {"error": f"{type(e).__name__}: {e}"}
     ck = clocks.stop()
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_decode(dec["wl"])
+        cpu = cpu_baseline_decode(dec["wl"], steps=5, warmup=1)
     value = whole_job_rate(dec["bytes"], dec["ms"], dist.world) / 1e9
     achieved = dec["bytes"] / (dec["ms"] * 1e-3) / 1e9
     peak = peaks["hbm_gbs"]

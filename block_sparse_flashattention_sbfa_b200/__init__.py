@@ -66,10 +66,12 @@ _SIGS = {
                                  _I, _I, _P, ctypes.c_size_t, T4, _P, _P, _P],
     "sbfa_varlen_selected_workspace_size": [_I, _I, _I, _I, _I, _I],
     "sbfa_check_status": [_P, _P],
+    "sbfa_set_wait_limit_ns": [ctypes.c_uint64],
     "sbfa_last_error": [],
     "sbfa_version": [],
 }
 _RESTYPES = {"sbfa_decode_workspace_size": ctypes.c_size_t,
+             "sbfa_set_wait_limit_ns": ctypes.c_uint64,
              "sbfa_varlen_selected_workspace_size": ctypes.c_size_t, "sbfa_last_error": ctypes.c_char_p,
              "sbfa_version": ctypes.c_char_p}
 
@@ -348,6 +350,13 @@ def fwd_varlen_selected(q, k, v, cu_seqlens, max_seqlen, sel, block=64, causal=T
 def check_status(status):
     """Synchronise and map the device status word to an exception."""
     _call("sbfa_check_status", _ptr(status), _stream())
+
+
+def set_wait_limit_ns(ns):
+    """Limit of the bounded waits inside the pipelined kernels launched from
+    now on (``sbfa_set_wait_limit_ns``; 0 restores the 2 s default).  Returns
+    the previous limit."""
+    return lib.sbfa_set_wait_limit_ns(int(ns))
 
 
 def new_status(device=None):

@@ -62,6 +62,7 @@ struct DecodeParams {
   const int* idx;
   int64_t tsb, tsh;
   int pair_mode;    // 1: every pair handled whole by one CTA (no workspace)
+  int dedup;        // 1: a block listed twice in a table row counts once
   int* ws_ticket;   // [B*Hkv]
   float* ws_part;   // [grid*2][rows][D]
   float* ws_lse;    // [grid*2][rows]
@@ -74,6 +75,7 @@ struct DecSmem {
   float mw[kDecGroupWarps][kDecRows];
   float lw[kDecGroupWarps][kDecRows];
   int2 meta[kDecWarps][kDecWarpStages];  // slice in each stage: {key0, nk | src << 7 | pr << 8}
+  uint32_t repeat[kDecWarps][2];         // repeat masks of a warp's even / odd chunk windows
   int last[2];                           // this CTA finishes shared pair 0 / 1
   // CTAs sharing this CTA's first / last pair: their partial slots (-1 for
   // an empty range) when there are at most kDecSharers of them, and count
@@ -213,13 +215,59 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     minfo = info;
   };
 
+  // With p.dedup, a table row that lists a block more than once counts it
+  // once: the chunks of every repeat after its first entry are skipped at
+  // compute time (their copies are still made).  Bit j % 32 of the window's mask in shared memory
+  // marks a repeat.  For each pair that the window's table chunks belong to,
+  // the warp reads the row's leading entries with one coalesced load per 32
+  // entries and every lane compares its own entry against the earlier ones
+  // by shuffles.  It runs after the window's first copies are issued, while
+  // they fly, and keeps nothing in registers across the streaming loop.
+  auto load_dup = [&](int win) {
+    const int j = win * 32 + lane;
+    int pr = 0, e = 0, jb = -1;
+    if (j < n_mine) {
+      const int64_t x = seq_x(grp + 2 * static_cast<int64_t>(j));
+      const int c = static_cast<int>(x % pp);
+      if (c >= nA) {
+        pr = static_cast<int>(x / pp);
+        e = (c - nA) / cpe;
+        jb = __ldg(p.idx + (pr / p.Hkv) * p.tsb + (pr % p.Hkv) * p.tsh + e);
+        if (jb >= p.n_kb) jb = -1;
+      }
+    }
+    bool dup = false;
+    uint32_t todo = __ballot_sync(0xffffffffu, jb >= 0);
+    while (todo) {
+      const int pr_l = __shfl_sync(0xffffffffu, pr, __ffs(todo) - 1);
+      const bool mine = jb >= 0 && pr == pr_l;
+      todo &= ~__ballot_sync(0xffffffffu, mine);
+      const int emax = static_cast<int>(__reduce_max_sync(0xffffffffu, mine ? e : 0));
+      const int* row = p.idx + (pr_l / p.Hkv) * p.tsb + (pr_l % p.Hkv) * p.tsh;
+      for (int c0 = 0; c0 < emax; c0 += 32) {
+        const int val = c0 + lane < emax ? __ldg(row + c0 + lane) : -1;
+        const int n = min(32, emax - c0);
+        for (int sl = 0; sl < n; ++sl) {
+          const int xv = __shfl_sync(0xffffffffu, val, sl);
+          dup |= mine && c0 + sl < e && xv == jb;
+        }
+      }
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, dup);
+    if (lane == 0) sm.repeat[warp][win & 1] = m;
+    __syncwarp();
+  };
+
   // Stream chunk j's slice of this warp into ring stage j % kDecWarpStages.
   // One commit group per call (empty past the end), so that "all but the
   // newest kDecWarpStages - 1 groups" is always the group of the oldest stage.
   auto issue = [&](int j) {
     const int stage = j % kDecWarpStages;
     if (j < n_mine) {
-      if ((j & 31) == 0 && j > 0) load_meta(j >> 5);
+      if ((j & 31) == 0 && j > 0) {
+        load_meta(j >> 5);
+        if (p.dedup) load_dup(j >> 5);
+      }
       const int key0 = __shfl_sync(0xffffffffu, mkey, j & 31);
       const int info = __shfl_sync(0xffffffffu, minfo, j & 31);
       if (lane == 0) sm.meta[warp][stage] = make_int2(key0, info);
@@ -288,6 +336,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   load_meta(0);
 #pragma unroll
   for (int s = 0; s < kDecWarpStages; ++s) issue(s);
+  if (p.dedup) load_dup(0);
 
   // While the first copies are in flight: which CTAs share this CTA's first
   // and last pair, and the partial slot each of them writes (the 64-bit
@@ -344,7 +393,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       const int stage = j % kDecWarpStages;
       const int2 mt = sm.meta[warp][stage];
       const int key0 = mt.x, nkeys = mt.y & 0x7f, src = (mt.y >> 7) & 1;
-      if (nkeys > kw) {
+      const bool repeat = p.dedup && ((sm.repeat[warp][(j >> 5) & 1] >> (j & 31)) & 1u);
+      if (nkeys > kw && !repeat) {
         const uint32_t kbase = smem_u32(sm.slice[warp][stage]);
         const uint32_t vbase = kbase + kDecSliceBytes / 2;
         float s[2][4];

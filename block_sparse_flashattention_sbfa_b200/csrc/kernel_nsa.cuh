@@ -53,6 +53,7 @@ struct NsaParams {
   int64_t oss, osh;
   float* lse;          // [Hq, total]
   int* status;
+  unsigned long long wait_ns;  // bounded-wait limit
 };
 
 __device__ __forceinline__ int nsa_seq_of(const int* cu, int nseq, int t) {
@@ -234,8 +235,9 @@ struct NsaSmem {
   alignas(16) float stage[8][32][32];
   uint32_t tmem_base;
   int abort_flag;
-  uint64_t k_full[2], v_full[2], q_full[2];
+  uint64_t k_full[2], v_full[2], q_full[2][2];  // q_full[buffer][producer warp]
   uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
 };
 
 struct NsaUnit {
@@ -293,11 +295,13 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.k_full[b], 1);
       mbar_init(&sm.v_full[b], 1);
-      mbar_init(&sm.q_full[b], 2);  // one expect-tx arrival per producer warp
+      mbar_init(&sm.q_full[b][0], 1);  // each producer warp arms its own half
+      mbar_init(&sm.q_full[b][1], 1);
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.p_full[b], 128);
       mbar_init(&sm.o_full[b], 1);
     }
+    mbar_init(&sm.mma_drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const WaitCtx wctx{&sm.abort_flag, p.status};
+  const WaitCtx wctx{&sm.abort_flag, p.status, p.wait_ns};
 
   if (warp == 0 || warp == 3) {
     // ===================== producers: Q rows by TMA gather4, K/V by TMA =====================
@@ -334,6 +338,10 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     }
     if (n_mine > 1) nxt = nsa_unit(p, u_lo + 1);
     bool ok = true;
+    // last unit whose Q (and, for warp 0, K) / V copies this warp issued into
+    // each buffer, for the drain before exit; a buffer is refilled only after
+    // its previous contents were consumed, so only that last phase can pend
+    int qk_last[2] = {-1, -1}, v_last[2] = {-1, -1};
     // Buffers of unit n (index n & 1) were last used by unit n - 2: Q and K
     // are free once QK(n - 2) has completed (s_full), V once PV(n - 2) has
     // (o_full), which comes after QK(n - 1) and so after Q(n - 1) landed.
@@ -349,7 +357,8 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       if (lane == 0) ok = mbar_wait(&sm.s_full[b], pw, wctx);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[b], 64 * 128 * 2);
+      qk_last[b] = n;
+      if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[b][half], 64 * 128 * 2);
       if (half == 0 && lane == 0) {
         mbar_arrive_expect_tx(&sm.k_full[b], kTileBytes);
         tma_load_4d(sm.k[b], &mapK, &sm.k_full[b], 0, cur.g, cur.key0, 0);
@@ -371,13 +380,14 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
           const int t = (code >= 0 ? code : first) / p.topk;
           y[i] = t * p.Hq + cur.g * p.G + r % p.G;
         }
-        tma_gather4_2d(sm.q[b] + colh * 16384 + (half * 64 + rl) * 128, &mapQ, &sm.q_full[b],
-                       colh * 64, y[0], y[1], y[2], y[3]);
+        tma_gather4_2d(sm.q[b] + colh * 16384 + (half * 64 + rl) * 128, &mapQ,
+                       &sm.q_full[b][half], colh * 64, y[0], y[1], y[2], y[3]);
       }
       if (half == 0) {
         if (lane == 0) {
           ok = mbar_wait(&sm.o_full[b], pw, wctx);
           if (ok) {
+            v_last[b] = n;
             mbar_arrive_expect_tx(&sm.v_full[b], kTileBytes);
             tma_load_4d(sm.v[b], &mapV, &sm.v_full[b], 0, cur.g, cur.key0, 0);
             tma_load_4d(sm.v[b] + 8192, &mapV, &sm.v_full[b], 64, cur.g, cur.key0, 0);
@@ -387,6 +397,18 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       }
       cur = nxt; nxt = nn;
       c0 = n0; c1 = n1; first = first_n;
+    }
+    // no copy may still be landing in shared memory when the CTA exits
+    __syncwarp();
+    if (lane == 0) {
+      for (int b = 0; b < 2; ++b) {
+        if (qk_last[b] >= 0) {
+          const uint32_t ph = (qk_last[b] >> 1) & 1;
+          mbar_wait_short(&sm.q_full[b][half], ph);
+          if (half == 0) mbar_wait_short(&sm.k_full[b], ph);
+        }
+        if (half == 0 && v_last[b] >= 0) mbar_wait_short(&sm.v_full[b], (v_last[b] >> 1) & 1);
+      }
     }
   } else if (warp == 1) {
     // ===================== MMA issuer =====================
@@ -403,7 +425,8 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
       auto issue_qk = [&](int n) -> bool {
         const int b = n & 1;
         const uint32_t ph = (n >> 1) & 1;
-        if (!mbar_wait(&sm.q_full[b], ph, wctx) || !mbar_wait(&sm.k_full[b], ph, wctx))
+        if (!mbar_wait(&sm.q_full[b][0], ph, wctx) || !mbar_wait(&sm.q_full[b][1], ph, wctx) ||
+            !mbar_wait(&sm.k_full[b], ph, wctx))
           return false;
         tc_fence_after();
         const uint64_t qd = qdesc0 + (b * kQTileBytes >> 4);
@@ -437,9 +460,10 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         if (n + 1 < n_mine) ok = issue_qk(n + 1);
         if (ok) ok = issue_pv(n);
       }
-      // drain every tcgen05 op before TMEM is released
-      umma_commit(&sm.s_full[0]);
-      mbar_wait_short(&sm.s_full[0], ((n_mine + 1) >> 1) & 1);
+      // drain every tcgen05 op before TMEM is released: a commit to a barrier
+      // nothing else uses completes its single phase only then
+      umma_commit(&sm.mma_drain);
+      mbar_wait_short(&sm.mma_drain, 0);
     }
     __syncwarp();
   } else if (warp >= 4) {

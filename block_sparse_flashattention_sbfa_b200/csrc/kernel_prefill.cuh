@@ -85,6 +85,7 @@ struct PrefillParams {
   const __nv_bfloat16* v;
   int64_t ksb, kss, ksh, vsb, vss, vsh;
   int* status;
+  unsigned long long wait_ns;  // bounded-wait limit
   unsigned long long* prof;  // 32 counters, self-profiling build only
 };
 
@@ -114,6 +115,7 @@ struct PfSmem {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
   uint64_t dec_full[kDecRingSlots], dec_empty[kDecRingSlots];
+  uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
 };
 
 static_assert(sizeof(PfSmem) + 1024 <= 232448, "prefill shared memory exceeds 227 KB");
@@ -330,6 +332,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.dec_full[i], 2);
       mbar_init(&sm.dec_empty[i], 1);
     }
+    mbar_init(&sm.mma_drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const WaitCtx wctx{&sm.abort_flag, p.status};
+  const WaitCtx wctx{&sm.abort_flag, p.status, p.wait_ns};
 
   if (warp == 0) {
     // ============================ Q/K producer ============================
@@ -358,6 +361,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     int ks = 0;
     uint32_t kph = 0;
+    // Armed phases, for the drain before exit: bit s of k_armed says stage s
+    // was ever filled, bit s of k_par holds the parity of its last fill; q_last
+    // is the last unit whose Q tiles were requested.  A stage is refilled only
+    // after its previous fill was consumed, so at most the last phase of each
+    // barrier can still be pending.
+    uint32_t k_armed = 0, k_par = 0;
+    int q_last = -1;
     bool ok = true;
     int n = 0;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
@@ -371,6 +381,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_arrive(&sm.sched_full[ub]);
         ok = mbar_wait_t(&sm.q_empty, (n & 1) ^ 1u, wctx, pacc[1]);
         if (ok) {
+          q_last = n;
           for (int t = 0; t < 2; ++t) {
             const int nv = sc.seg_valid[2 * t] + sc.seg_valid[2 * t + 1];
             mbar_arrive_expect_tx(&sm.q_full[t], nv * 2 * 8192);
@@ -392,6 +403,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
         if (!good) return false;
         const int halves = (mem | (mem >> 2) | (mem >> 4) | (mem >> 6)) & 3;
+        k_armed |= 1u << ks;
+        k_par = (k_par & ~(1u << ks)) | (kph << ks);
         if (!has_cols || !is_col) {
           if (lane == 0) {
             mbar_arrive_expect_tx(&sm.k_full[ks], __popc(halves) * 2 * 8192);
@@ -413,12 +426,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       };
       ok = pf_for_each<has_cols>(sc, body);
     }
-    if (!ok && lane == 0)
-      for (int i = 0; i < kKStages; ++i) mbar_wait_short(&sm.k_full[i], 0);
+    // no copy may still be landing in shared memory when the CTA exits
+    if (lane == 0) {
+      for (int i = 0; i < kKStages; ++i)
+        if ((k_armed >> i) & 1) mbar_wait_short(&sm.k_full[i], (k_par >> i) & 1);
+      if (q_last >= 0)
+        for (int t = 0; t < 2; ++t) mbar_wait_short(&sm.q_full[t], q_last & 1);
+    }
   } else if (warp == 2) {
     // ============================= V producer =============================
     int vs = 0;
     uint32_t vph = 0;
+    uint32_t v_armed = 0, v_par = 0;  // as k_armed / k_par above
     int dslot = 0;
     uint32_t dph = 0;
     bool ok = true;
@@ -449,6 +468,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (lane == 0) good = mbar_wait_t(&sm.v_empty[vs], vph ^ 1u, wctx, pacc[0]);
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
         if (!good) return false;
+        v_armed |= 1u << vs;
+        v_par = (v_par & ~(1u << vs)) | (vph << vs);
         if (!has_cols || !is_col) {
           if (lane == 0) {
             mbar_arrive_expect_tx(&sm.v_full[vs], __popc(need) * 2 * 8192);
@@ -472,8 +493,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sched_empty[ub]);
     }
-    if (!ok && lane == 0)
-      for (int i = 0; i < kVStages; ++i) mbar_wait_short(&sm.v_full[i], 0);
+    if (lane == 0)
+      for (int i = 0; i < kVStages; ++i)
+        if ((v_armed >> i) & 1) mbar_wait_short(&sm.v_full[i], (v_par >> i) & 1);
   } else if (warp == 1) {
     // ============================= MMA issuer =============================
     if (lane == 0) {
@@ -595,9 +617,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         umma_commit(&sm.q_empty);
         mbar_arrive(&sm.sched_empty[ub]);
       }
-      // every issued tcgen05 op must finish before TMEM is freed
-      umma_commit(&sm.q_empty);
-      mbar_wait_short(&sm.q_empty, (n & 1));
+      // every issued tcgen05 op must finish before TMEM is freed: a commit
+      // to a barrier nothing else uses completes its single phase only then
+      umma_commit(&sm.mma_drain);
+      mbar_wait_short(&sm.mma_drain, 0);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -621,6 +644,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int ub = n & 1;
       PfSched& sc = sm.sched[ub];
       ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
+      // gated mode synchronises the warpgroup on named barriers: its four
+      // warps must leave together, so every exit is agreed on one first
+      if (gated) ok = !named_bar_or(bar_id, 128, !ok);
       if (!ok) break;
       const int my_valid = sc.seg_valid[seg];
       const int my_row = sc.seg_row0[seg] + (r & 63);
@@ -807,8 +833,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int head = sc.seg_head[seg];
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       if (npv > 0) {
-        const bool okd = __all_sync(0xffffffffu,
-                                    mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1]));
+        bool okd = __all_sync(0xffffffffu,
+                              mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1]));
+        if (gated) okd = !named_bar_or(bar_id, 128, !okd);  // npv is uniform in the warpgroup
         if (!okd) { ok = false; break; }
         tc_fence_after();
         float ob[32];

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -162,6 +163,10 @@ float eff_scale(const sbfa_shape* s) {
 // sbfa_set_profile_counters, which only that build exports.
 unsigned long long* g_prof_counters = nullptr;
 
+// Limit of the kernels' bounded waits, read at every launch
+// (sbfa_set_wait_limit_ns).
+std::atomic<unsigned long long> g_wait_ns{sbfa::kWaitLimitNs};
+
 // ---------------------------------------------------------------------------
 // prefill launcher (tcgen05 kernel)
 // ---------------------------------------------------------------------------
@@ -213,6 +218,7 @@ sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sb
     attr_set[dev][p.mode] = true;
   }
   p.prof = g_prof_counters;
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   const int grid = std::min(p.n_units, di.sms);
   switch (p.mode) {
     case sbfa::kModeTable:
@@ -434,7 +440,11 @@ extern "C" {
 
 const char* sbfa_last_error(void) { return g_last_error.c_str(); }
 
-const char* sbfa_version(void) { return "sbfa 0.1 (sm_100a)"; }
+const char* sbfa_version(void) { return "sbfa 0.2 (sm_100a)"; }
+
+uint64_t sbfa_set_wait_limit_ns(uint64_t ns) {
+  return g_wait_ns.exchange(ns ? ns : sbfa::kWaitLimitNs);
+}
 
 #ifdef SBFA_PROFILE
 // Self-profiling build only: device array of 33 uint64 counters that the
@@ -459,6 +469,7 @@ sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
   SBFA_TRY(check_table(table, shape, !dec));
   if (dec) {
     sbfa::DecodeParams p{};
+    p.dedup = 1;  // a row is a set of blocks, as on the tiled kernel
     return launch_decode(p, shape, q, nullptr, nullptr, 0, 0, &k, &v, table, nullptr, 0, o,
                          lse, status, reinterpret_cast<cudaStream_t>(stream));
   }
@@ -760,6 +771,7 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   p.o = static_cast<__nv_bfloat16*>(o.ptr); p.oss = o.ss; p.osh = o.sh;
   p.lse = lse;
   p.status = status;
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   const int64_t nb = static_cast<int64_t>(Hkv) * nseq * p.nbps;
   if (nb > (1 << 26)) return fail(SBFA_ERR_UNSUPPORTED, "too many key blocks");
   CUtensorMap mq, mk, mv;

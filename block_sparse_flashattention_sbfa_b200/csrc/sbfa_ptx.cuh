@@ -14,7 +14,8 @@ constexpr int kDevBadIndex = 0x1;
 constexpr int kDevTimeout = 0x2;
 constexpr int kDevOverflow = 0x4;
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
+// By default a bounded wait gives up after this many nanoseconds of
+// %globaltimer; a launch may carry a different limit (sbfa_set_wait_limit_ns).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -76,20 +77,56 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 struct WaitCtx {
   volatile int* abort_flag;  // shared memory
   int* status;               // global, may be null
+  uint64_t limit_ns;         // give up after this long
 };
+
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Short-limit variant of mbar_wait below: polls with the non-suspending
+// test_wait and looks at the clock on every poll, so that limits on the
+// nanosecond scale are kept.  Out of line: it is only reached when a launch
+// carries such a limit, and it keeps the inlined wait small.
+__device__ __noinline__ bool mbar_wait_poll(uint32_t addr, uint32_t parity, volatile int* abort_flag,
+                                            int* status, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_test_wait(addr, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      report(status, kDevTimeout);
+      return false;
+    }
+  }
+  return true;
+}
 
 // Wait until the phase with the given parity has completed.  Returns false
 // (after raising the CTA's abort flag and the device status bit) if the wait
-// exceeds kWaitLimitNs, or if another role of the CTA already aborted.
+// exceeds ctx.limit_ns, or if another role of the CTA already aborted.  The
+// suspending try_wait polls; the abort flag and the clock are looked at every
+// 256 polls (limits under a millisecond go to mbar_wait_poll instead).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
-  uint64_t t0 = globaltimer();
+  if (ctx.limit_ns < 1000000ull)
+    return mbar_wait_poll(addr, parity, ctx.abort_flag, ctx.status, ctx.limit_ns);
+  const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 255u) == 0) {
       if (*ctx.abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > ctx.limit_ns) {
         *ctx.abort_flag = 1;
         report(ctx.status, kDevTimeout);
         return false;
@@ -120,7 +157,10 @@ __device__ __forceinline__ bool mbar_wait_t(uint64_t* bar, uint32_t parity, cons
 #endif
 }
 
-// Short bounded wait used only on abort paths (drain in-flight copies).
+// Bounded wait used only to drain a CTA's own in-flight copies or MMAs
+// before it exits (whatever the abort state).  The caller passes the parity
+// of the last phase it armed; it must know that no earlier phase of the
+// barrier is still pending, or the parity test would see that older phase.
 __device__ __forceinline__ void mbar_wait_short(uint64_t* bar, uint32_t parity) {
   const uint32_t addr = smem_u32(bar);
   uint64_t t0 = globaltimer();

@@ -71,10 +71,11 @@ typedef struct {
  * generalised per (batch, kv-head, q-block)).  Row r of query head h in
  * batch b uses idx[b*sb + (h/G)*sh + (r/q_block)*sqb + n], n < nmax.  Each
  * entry j >= 0 names the keys [j*kv_block, (j+1)*kv_block) clipped to Sk;
- * entries < 0 are padding; order does not matter.  A row must list each
- * block at most once (a repeat is a precondition violation: the split-KV
- * kernel would count it twice, the tiled kernel once).  sb = sh = sqb = 0
- * broadcasts one 1-D table (the README's form).
+ * entries < 0 are padding; order does not matter; a row is a set of blocks:
+ * sbfa_fwd counts a block listed more than once once, whichever kernel
+ * serves the call (see sbfa_speculative_sparse for its own rule).  An entry
+ * >= ceil(Sk / kv_block) is skipped and sets SBFA_DEV_BAD_INDEX.
+ * sb = sh = sqb = 0 broadcasts one 1-D table (the README's form).
  */
 typedef struct {
   const int32_t* idx;
@@ -145,6 +146,9 @@ sbfa_status sbfa_combine(int32_t n_parts, int32_t B, int32_t Sq, int32_t Hq, int
  * sequences (batch stride 0), kv_block = the page size, and each table row
  * listing the pool pages of its missed blocks (FlagAttention's paged
  * attention; pages may be shared between sequences).
+ * `missed` lists distinct blocks (README, Usage 2: the blocks the
+ * speculative pass missed); the fused kernel does not look for repeats, so
+ * a block listed twice would be counted twice.
  * Limits: Sq * (Hq/Hkv) <= 16; missed->q_block >= Sq; missed->kv_block in
  * {16, 32, 64, 128, 256}; B*Hkv <= 4096; missed->nmax <= 1024.
  * ws/ws_bytes: device workspace of at least sbfa_decode_workspace_size()
@@ -296,6 +300,21 @@ sbfa_status sbfa_check_status(const int32_t* status, sbfa_stream_t stream);
  */
 sbfa_status sbfa_calibrate_thresholds(const float* smax, int32_t B, int32_t Hq, int32_t n_qb,
                                       int32_t k_top, float* T, sbfa_stream_t stream);
+
+/*
+ * sbfa_set_wait_limit_ns -- time limit of the bounded waits inside the
+ * pipelined kernels (sbfa_fwd's tiled path, sbfa_fwd_dense, sbfa_fwd_partials,
+ * sbfa_fwd_gated, sbfa_fwd_vertical_slash, sbfa_fwd_varlen_selected)
+ * launched after the call, for the whole process.  No wait in these kernels
+ * is unbounded: one that runs past the limit stops its CTA early (every
+ * copy and tensor-core operation the CTA issued is drained first, so the
+ * context stays usable) and sets SBFA_DEV_TIMEOUT in the status word, and
+ * sbfa_check_status then returns SBFA_ERR_TIMEOUT; the outputs of that
+ * launch are incomplete.  0 restores the default of 2 s.  Returns the
+ * previous limit.  The split-KV decode kernel and the index kernels have no
+ * waits and ignore it.
+ */
+uint64_t sbfa_set_wait_limit_ns(uint64_t ns);
 
 /* Message of the last error on this host thread ("" if none). */
 const char* sbfa_last_error(void);

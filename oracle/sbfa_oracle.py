@@ -319,7 +319,7 @@ def kept_density_closed_form(n, k_top):
 # ----------------------------------------------------------------------------
 
 def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
-                           block_M, block_N, causal=True):
+                           block_M, block_N, causal=True, qblocks=None):
     """Per (b, h, q-block i), rows [m0, m1) with m1 = min(m0 + BM, q_len):
 
     * a slash offset s is the diagonal key = row + (kv_len - q_len) - s; over
@@ -330,7 +330,9 @@ def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
     * column_index = ascending vertical columns v < kv_len (and, if causal,
       v <= m1-1+d) that lie in no listed block, column_count = their number.
     Entries past the counts are 0.  (Sglang Sparse Flash Attention, I/O
-    contract; the aligned-block reading is an assumption.)"""
+    contract; the aligned-block reading is an assumption.)  ``qblocks``:
+    None (every q-block) or the q-block indices to convert; the others are
+    left at count 0."""
     B, H, nnz_v = vertical.shape
     nnz_s = slash.shape[2]
     nqb = -(-context_size // block_M)
@@ -345,7 +347,7 @@ def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
         for h in range(H):
             s = slash[b, h].astype(np.int64)
             vv = vertical[b, h].astype(np.int64)
-            for i in range(nqb):
+            for i in (range(nqb) if qblocks is None else qblocks):
                 m0 = i * block_M
                 if m0 >= ql:
                     continue

@@ -114,3 +114,43 @@ def test_oracle_samples_beside_the_prefill_numbers():
     for line in (g, v, n):
         assert line["kind"] == "oracle" and line["value"] > 0 and line["sample_seconds"] > 0
         assert line["extrapolated_full_seconds"] > line["sample_seconds"]
+    c = bm.oracle_sample_vs_convert(wv, n_qb=4)
+    assert c["extrapolated_full_seconds"] >= c["sample_seconds"] > 0
+
+
+def test_oracle_sample_flops_match_element_counts():
+    """The FLOPs each oracle sample line divides by, against element-by-element
+    counts of the pairs that sample evaluates."""
+    bm = _bench()
+    # gated: q-block i of one head; QK over every causal key, PV over kept blocks
+    rng = np.random.default_rng(21)
+    L, i = 640, 9
+    keep = rng.random(i + 1) < 0.5
+    keep[i] = True
+    r = np.arange(i * 64, (i + 1) * 64)
+    qk = int((np.arange(L)[None, :] <= r[:, None]).sum())
+    kept_keys = np.concatenate([np.arange(j * 64, (j + 1) * 64) for j in np.nonzero(keep)[0]])
+    pv = int((kept_keys[None, :] <= r[:, None]).sum())
+    assert bm.gated_sample_flops(i, keep) == 2 * 128 * (qk + pv)
+    # vertical/slash: visible pairs of one q-block under converted lists
+    L = 1024
+    vert, slash = W.vertical_slash_indices(np.random.default_rng(22), 1, 1, L, 80, 120)
+    bc, bo, cc, ci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    for i in (3, 15):
+        rows = np.arange(i * 64, (i + 1) * 64)
+        keys = set()
+        for off in bo[0, 0, i, :bc[0, 0, i]]:
+            keys.update(range(off, min(off + 64, L)))
+        keys.update(int(c) for c in ci[0, 0, i, :cc[0, 0, i]])
+        kk = np.array(sorted(keys))
+        assert bm.vs_sample_pairs(bc, bo, cc, ci, i, L) == int((kk[None, :] <= rows[:, None]).sum())
+    # NSA: visible pairs of head 0 over chosen tokens of sequence 0
+    wl = W.make_nsa_varlen(seqlens=(500, 100), H=2, seed=23, table_seed=24)
+    cu, sel = wl.meta["cu_seqlens"], wl.meta["sel"]
+    toks = np.arange(400, 500)
+    count = 0
+    for t in toks:
+        for j in sel[t, 0]:
+            if j >= 0:
+                count += max(0, min(64, t - 64 * int(j) + 1))
+    assert bm.nsa_sample_pairs(cu, sel, toks) == count

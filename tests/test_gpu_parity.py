@@ -222,6 +222,34 @@ def test_block_table_short_queries(sb, Sq, G, causal):
     compare(o, lse, ro, rl, f"short queries Sq={Sq} G={G} causal={causal}")
 
 
+def test_repeated_blocks_count_once_on_split_kv(sb):
+    """A table row that lists a block more than once counts it once in
+    sbfa_fwd whichever kernel serves the call: with one query position it
+    runs on the split-KV kernel, with 64 on the tiled one; both against the
+    oracle's set reading of a table row."""
+    rng = np.random.default_rng(311)
+    B, Hq, Hkv, Sk, bs, nmax = 2, 8, 2, 2000, 64, 12
+    nkb = -(-Sk // bs)
+    tab = np.full((B, Hkv, 1, nmax), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            first = rng.choice(nkb, size=7, replace=False)
+            row = np.concatenate([first, rng.choice(first, size=3), [-1, -1]])
+            rng.shuffle(row)
+            tab[b, g, 0] = row
+    assert any(len(set(r[r >= 0])) < (r >= 0).sum() for r in tab.reshape(-1, nmax))
+    k = W.normal_bf16(rng, (B, Sk, Hkv, 128))
+    v = W.normal_bf16(rng, (B, Sk, Hkv, 128))
+    td = torch.from_numpy(tab).cuda()
+    for Sq in (1, 64):
+        q = W.normal_bf16(rng, (B, Sq, Hq, 128))
+        st = sb.new_status("cuda")
+        o, lse = sb.fwd(dev(q), dev(k), dev(v), td, Sq, bs, causal=False, status=st)
+        sb.check_status(st)
+        ro, rl = oracle.attend_block_table(q, k, v, tab, Sq, bs, False, W.default_scale())
+        compare(o, lse, ro, rl, f"repeats, sbfa_fwd Sq={Sq}")
+
+
 def test_paged_kv_decode(sb):
     """A paged KV cache through the same entry point: one physical pool of
     pages shared by every sequence (k/v views with batch stride 0), each
@@ -266,9 +294,12 @@ def _gated_small(L=1024, Hq=8, Hkv=2, k_top=4):
 
 
 def _check_keep(info, smax_g, keep_g, T, what):
-    """Keep bits bit-exact except blocks whose s_max is within 1e-3 of T."""
+    """Keep bits bit-exact except blocks whose s_max is within 1e-3 of T,
+    which are reported.  Returns the (b, h, i) q-blocks that hold such a
+    near-threshold flip."""
     n_diff = n_near = n_tot = 0
     max_sm_err = 0.0
+    flipped = []
     for (b, h, i), (sm_ref, keep_ref) in info.items():
         kg = keep_g[b, h, i, :i + 1].astype(bool)
         sg = smax_g[b, h, i, :i + 1]
@@ -278,11 +309,33 @@ def _check_keep(info, smax_g, keep_g, T, what):
         n_near += int((diff & near).sum())
         n_diff += int((diff & ~near).sum())
         n_tot += i + 1
+        if (diff & near).any():
+            flipped.append((b, h, i))
+            print(f"{what}: near-threshold flip at b={b} h={h} i={i}, blocks "
+                  f"{np.nonzero(diff & near)[0].tolist()}")
     print(f"{what}: {n_tot} blocks, keep mismatches {n_diff}, near-threshold flips {n_near}, "
           f"s_max max-abs {max_sm_err:.2e}")
     assert n_diff == 0
     assert max_sm_err < 1e-3
-    return n_near
+    return flipped
+
+
+def _regate(wl, keep_g, flipped, ro, rl, block=64):
+    """For a q-block whose keep row differs from the oracle's only by
+    near-threshold flips, the oracle's output rows are recomputed over the
+    blocks the GPU kept, so that every sampled row is still compared."""
+    L = wl.q.shape[1]
+    G = wl.q.shape[2] // wl.k.shape[2]
+    for (b, h, i) in flipped:
+        kept = np.nonzero(keep_g[b, h, i, :i + 1])[0]
+        keys = (kept[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+        keys = keys[keys < L]
+        r = np.arange(i * block, min((i + 1) * block, L))
+        oo, ll = oracle.attend_keyset(wl.q[b, r, h, :], wl.k[b, keys, h // G, :],
+                                      wl.v[b, keys, h // G, :], keys[None, :] <= r[:, None],
+                                      wl.scale)
+        ro[b, r, h, :] = oo
+        rl[b, h, r] = ll
 
 
 def test_gated_small_all_rows(sb):
@@ -293,11 +346,30 @@ def test_gated_small_all_rows(sb):
     keep = torch.full((1, 8, n, n), 255, dtype=torch.uint8, device="cuda")
     o, lse = sb.fwd_gated(q, k, v, torch.from_numpy(T).cuda(), smax_out=smax, keep_out=keep)
     ro, rl, info = oracle.attend_gated(wl.q, wl.k, wl.v, T, 64, wl.scale, return_keep=True)
-    near = _check_keep(info, smax.cpu().numpy(), keep.cpu().numpy(), T, "gated small")
-    if near == 0:
-        compare(o, lse, ro, rl, "gated small")
     kept = keep.cpu().numpy()
+    flipped = _check_keep(info, smax.cpu().numpy(), kept, T, "gated small")
+    _regate(wl, kept, flipped, ro, rl)
+    compare(o, lse, ro, rl, "gated small")
     assert np.all(kept[0][:, np.triu_indices(n, 1)[0], np.triu_indices(n, 1)[1]] == 255)
+
+
+@pytest.mark.parametrize("L", [1000, 1090])
+def test_gated_ragged_length(sb, L):
+    """A sequence length that is not a multiple of 64: the last q-block and
+    the last key block are partial (all rows checked)."""
+    wl, T = _gated_small(L=L, Hq=8, Hkv=2, k_top=3)
+    n = T.shape[1]
+    smax = torch.full((1, 8, n, n), float("nan"), device="cuda")
+    keep = torch.full((1, 8, n, n), 255, dtype=torch.uint8, device="cuda")
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_gated(dev(wl.q), dev(wl.k), dev(wl.v), torch.from_numpy(T).cuda(),
+                          smax_out=smax, keep_out=keep, status=st)
+    sb.check_status(st)
+    ro, rl, info = oracle.attend_gated(wl.q, wl.k, wl.v, T, 64, wl.scale, return_keep=True)
+    kept = keep.cpu().numpy()
+    flipped = _check_keep(info, smax.cpu().numpy(), kept, T, f"gated L={L}")
+    _regate(wl, kept, flipped, ro, rl)
+    compare(o, lse, ro, rl, f"gated L={L}")
 
 
 def test_gated_full_workload_sampled(sb):
@@ -316,12 +388,12 @@ def test_gated_full_workload_sampled(sb):
     ro, rl, info = oracle.attend_gated(wl.q, wl.k, wl.v, T, 64, wl.scale,
                                        rows=lambda b, h: rows[h], return_keep=True)
     kp = keep.cpu().numpy()
-    near = _check_keep(info, smax.cpu().numpy(), kp, T, "gated full")
+    flipped = _check_keep(info, smax.cpu().numpy(), kp, T, "gated full")
     dens = sum(int(kp[0, h, i, :i + 1].sum()) for (_, h, i) in info) / \
         sum(i + 1 for (_, _, i) in info)
     print(f"gated full: kept density on the sampled q-blocks {dens:.3f}")
-    if near == 0:
-        compare(o, lse, ro, rl, "gated full")
+    _regate(wl, kp, flipped, ro, rl)
+    compare(o, lse, ro, rl, "gated full")
 
 
 def test_calibrate_thresholds_exact(sb):
@@ -400,9 +472,10 @@ def test_vertical_slash_columns_heavy(sb):
 
 def test_vertical_slash_full_workload_sampled(sb):
     """L=131072, H=32, 1000 vertical columns and 6000 slash offsets per head,
-    64 x 64 blocks, causal.  The GPU's converted lists match the oracle's bit
-    for bit on every q-block of 8 heads, and on those heads 4 whole q-blocks
-    (256 rows, always including the last) match the oracle's attention."""
+    64 x 64 blocks, causal.  On every one of the 32 heads, 4 whole seeded
+    q-blocks (256 rows, always including the last): the GPU's converted lists
+    match the oracle's bit for bit, and the attention rows match the
+    oracle's."""
     wl = W.make_vertical_slash()
     L, H = wl.q.shape[1], wl.q.shape[2]
     vert, slash = wl.meta["vertical"], wl.meta["slash"]
@@ -411,22 +484,85 @@ def test_vertical_slash_full_workload_sampled(sb):
                                                torch.from_numpy(slash).cuda(), L)
     o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), bc, bo, cc, ci, causal=True)
     torch.cuda.synchronize()
-    heads = [0, 5, 11, 17, 22, 26, 29, 31]
-    hi = torch.tensor(heads, device="cuda")
-    gbc, gbo, gcc, gci = (x.index_select(1, hi).cpu().numpy() for x in (bc, bo, cc, ci))
-    del bo, ci
-    ref = [oracle.convert_vertical_slash([L], [L], vert[:, h:h + 1], slash[:, h:h + 1], L, 64,
-                                         64, True) for h in heads]
-    rbc, rbo, rcc, rci = (np.concatenate([r[i] for r in ref], axis=1) for i in range(4))
-    assert np.array_equal(gbc, rbc) and np.array_equal(gcc, rcc)
-    for idx in np.ndindex(rbc.shape):
-        assert np.array_equal(gbo[idx][:rbc[idx]], rbo[idx][:rbc[idx]])
-        assert np.array_equal(gci[idx][:rcc[idx]], rci[idx][:rcc[idx]])
-    rows = {j: sampled_rows(L, 64, 700 + h) for j, h in enumerate(heads)}
-    ro, rl = oracle.attend_vertical_slash(wl.q[:, :, heads], wl.k[:, :, heads], wl.v[:, :, heads],
-                                          rbc, rbo, rcc, rci, 64, 64, True, wl.scale,
-                                          rows=lambda b, j: rows[j])
-    compare(o[:, :, heads], lse[:, heads], ro, rl, "vs full")
+    n_rows = n_lists = 0
+    err_o = err_l = 0.0
+    for h in range(H):
+        qbs = W.sample_qblocks(np.random.default_rng(700 + h), L // 64)
+        rbc, rbo, rcc, rci = oracle.convert_vertical_slash([L], [L], vert[:, h:h + 1],
+                                                           slash[:, h:h + 1], L, 64, 64, True,
+                                                           qblocks=qbs)
+        qi = torch.from_numpy(qbs).cuda()
+        gbc, gcc = (x[0, h].index_select(0, qi).cpu().numpy() for x in (bc, cc))
+        gbo, gci = (x[0, h].index_select(0, qi).cpu().numpy() for x in (bo, ci))
+        for j, i in enumerate(qbs):
+            assert gbc[j] == rbc[0, 0, i] and gcc[j] == rcc[0, 0, i], (h, i)
+            assert np.array_equal(gbo[j][:gbc[j]], rbo[0, 0, i][:rbc[0, 0, i]]), (h, i)
+            assert np.array_equal(gci[j][:gcc[j]], rci[0, 0, i][:rcc[0, 0, i]]), (h, i)
+            n_lists += 1
+        rows = np.concatenate([np.arange(i * 64, (i + 1) * 64) for i in qbs])
+        ro, rl = oracle.attend_vertical_slash(wl.q[:, :, h:h + 1], wl.k[:, :, h:h + 1],
+                                              wl.v[:, :, h:h + 1], rbc, rbo, rcc, rci, 64, 64,
+                                              True, wl.scale, rows=lambda b, j: rows)
+        ri = torch.from_numpy(rows).cuda()
+        og = o[0, :, h].index_select(0, ri).float().cpu().numpy()
+        lg = lse[0, h].index_select(0, ri).cpu().numpy()
+        assert np.isfinite(lg).all()
+        err_o = max(err_o, np.abs(og - ro[0, rows, 0]).max())
+        err_l = max(err_l, np.abs(lg - rl[0, 0, rows]).max())
+        n_rows += rows.size
+    print(f"vs full: {n_lists} converted q-blocks exact, {n_rows} rows on {H} heads, "
+          f"o max-abs {err_o:.3e}, lse max-abs {err_l:.3e}")
+    assert err_o <= O_TOL and err_l <= LSE_TOL
+
+
+def test_vertical_slash_ragged_length(sb):
+    """L = 1500 (partial last q-block and key block), all rows checked."""
+    wl = _vs_small(L=1500, H=2, nnz_v=80, nnz_s=120, seed=42)
+    L = wl.q.shape[1]
+    vert, slash = wl.meta["vertical"], wl.meta["slash"]
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    bc, bo, cc, ci = sb.convert_vertical_slash(sl, sl, torch.from_numpy(vert).cuda(),
+                                               torch.from_numpy(slash).cuda(), L)
+    rbc, rbo, rcc, rci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    _check_lists((bc, bo, cc, ci), (rbc, rbo, rcc, rci))
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), bc, bo, cc, ci, causal=True,
+                                   status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, rbc, rbo, rcc, rci, 64, 64, True,
+                                          wl.scale)
+    compare(o, lse, ro, rl, "vs L=1500")
+
+
+def test_vertical_slash_batch2_short_queries(sb):
+    """B = 2 with q_len = 700 < kv_len = 1000 (bottom-right causal alignment:
+    slash offsets and the causal limit are shifted by kv_len - q_len)."""
+    rng = np.random.default_rng(43)
+    B, H, Sq, Sk = 2, 2, 700, 1000
+    q = W.normal_bf16(rng, (B, Sq, H, 128))
+    k = W.normal_bf16(rng, (B, Sk, H, 128))
+    v = W.normal_bf16(rng, (B, Sk, H, 128))
+    vert, slash = W.vertical_slash_indices(np.random.default_rng(1043), B, H, Sk, 70, 90)
+    qs = torch.tensor([Sq] * B, dtype=torch.int32, device="cuda")
+    ks = torch.tensor([Sk] * B, dtype=torch.int32, device="cuda")
+    bc, bo, cc, ci = sb.convert_vertical_slash(qs, ks, torch.from_numpy(vert).cuda(),
+                                               torch.from_numpy(slash).cuda(), Sq)
+    rbc, rbo, rcc, rci = oracle.convert_vertical_slash([Sq] * B, [Sk] * B, vert, slash, Sq, 64,
+                                                       64, True)
+    _check_lists((bc, bo, cc, ci), (rbc, rbo, rcc, rci))
+    o, lse = sb.fwd_vertical_slash(dev(q), dev(k), dev(v), bc, bo, cc, ci, causal=True)
+    ro, rl = oracle.attend_vertical_slash(q, k, v, rbc, rbo, rcc, rci, 64, 64, True,
+                                          W.default_scale())
+    compare(o, lse, ro, rl, "vs B=2 Sq<Sk")
+
+
+def _check_lists(gpu, ref):
+    bc, bo, cc, ci = (x.cpu().numpy() for x in gpu)
+    rbc, rbo, rcc, rci = ref
+    assert np.array_equal(bc, rbc) and np.array_equal(cc, rcc)
+    for idx in np.ndindex(bc.shape):
+        assert np.array_equal(bo[idx][:bc[idx]], rbo[idx][:rbc[idx]])
+        assert np.array_equal(ci[idx][:cc[idx]], rci[idx][:rcc[idx]])
 
 
 # ------------------------------------------------------------------ NSA selected (varlen)

@@ -1,11 +1,13 @@
 """The allocation-free decode entry point (fixed scratch compiled into the
 library, for callers that cannot call cudaMalloc) must give the results of
-the workspace entry point, on two calls in a row (the second call reuses
-the scratch the first one left behind).  Collected last on purpose."""
+the workspace entry point, and match the fp64 oracle, on two calls in a row
+(the second call reuses the scratch the first one left behind).  Collected
+last on purpose."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -29,6 +31,8 @@ def test_noalloc_matches_workspace_entry_point(sb, shape):
     q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
     tab = torch.from_numpy(wl.meta["table"]).cuda()
     ref_o, ref_l = sb.speculative_sparse(q, k[:, s0:], v[:, s0:], True, k, v, tab, 128)
+    oo, ol = oracle.speculative_sparse(wl.q, wl.k[:, s0:], wl.v[:, s0:], True, wl.k, wl.v,
+                                       wl.meta["table"], 128, wl.scale)
     st = sb.new_status("cuda")
     out = torch.empty_like(q)
     lse = torch.empty_like(ref_l)
@@ -40,8 +44,12 @@ def test_noalloc_matches_workspace_entry_point(sb, shape):
         sb.check_status(st)
         eo = (out.float() - ref_o.float()).abs().max().item()
         el = (lse - ref_l).abs().max().item()
-        print(f"no-alloc call {call}: o max-abs {eo:.2e}, lse max-abs {el:.2e}")
+        ro = np.abs(out.float().cpu().numpy() - oo).max()
+        rl = np.abs(lse.cpu().numpy() - ol).max()
+        print(f"no-alloc call {call}: vs workspace path o {eo:.2e} lse {el:.2e}; "
+              f"vs oracle o {ro:.2e} lse {rl:.2e}")
         assert eo <= 2e-2 and el <= 1e-3
+        assert ro <= 2e-2 and rl <= 1e-3
 
 
 def test_noalloc_rejects_too_many_pairs(sb):
