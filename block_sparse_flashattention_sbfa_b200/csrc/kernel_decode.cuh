@@ -62,7 +62,6 @@ struct DecodeParams {
   const int* idx;
   int64_t tsb, tsh;
   int pair_mode;    // 1: every pair handled whole by one CTA (no workspace)
-  int dedup;        // 1: a block listed twice in a table row counts once
   int* ws_ticket;   // [B*Hkv]
   float* ws_part;   // [grid*2][rows][D]
   float* ws_lse;    // [grid*2][rows]
@@ -132,6 +131,9 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
+// DEDUP: a block listed more than once in a table row counts once (the
+// repeat scan below); without it the kernel trusts the rows to be sets.
+template <bool DEDUP>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     minfo = info;
   };
 
-  // With p.dedup, a table row that lists a block more than once counts it
+  // With DEDUP, a table row that lists a block more than once counts it
   // once: the chunks of every repeat after its first entry are skipped at
   // compute time (their copies are still made).  Bit j % 32 of the window's mask in shared memory
   // marks a repeat.  For each pair that the window's table chunks belong to,
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     if (j < n_mine) {
       if ((j & 31) == 0 && j > 0) {
         load_meta(j >> 5);
-        if (p.dedup) load_dup(j >> 5);
+        if (DEDUP) load_dup(j >> 5);
       }
       const int key0 = __shfl_sync(0xffffffffu, mkey, j & 31);
       const int info = __shfl_sync(0xffffffffu, minfo, j & 31);
@@ -336,7 +338,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
   load_meta(0);
 #pragma unroll
   for (int s = 0; s < kDecWarpStages; ++s) issue(s);
-  if (p.dedup) load_dup(0);
+  if (DEDUP) load_dup(0);
 
   // While the first copies are in flight: which CTAs share this CTA's first
   // and last pair, and the partial slot each of them writes (the 64-bit
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       const int stage = j % kDecWarpStages;
       const int2 mt = sm.meta[warp][stage];
       const int key0 = mt.x, nkeys = mt.y & 0x7f, src = (mt.y >> 7) & 1;
-      const bool repeat = p.dedup && ((sm.repeat[warp][(j >> 5) & 1] >> (j & 31)) & 1u);
+      const bool repeat = DEDUP && ((sm.repeat[warp][(j >> 5) & 1] >> (j & 31)) & 1u);
       if (nkeys > kw && !repeat) {
         const uint32_t kbase = smem_u32(sm.slice[warp][stage]);
         const uint32_t vbase = kbase + kDecSliceBytes / 2;

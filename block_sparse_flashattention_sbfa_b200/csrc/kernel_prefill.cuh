@@ -5,9 +5,7 @@
 //               key-tile schedule in shared memory; gathers K rows of
 //               vertical columns
 //   warp 1      tcgen05 MMA issuer (one lane); owns the TMEM allocation
-//   warp 2      producer for V tiles -- in gated mode it waits for the
-//               gate's keep decision and loads no V for pruned blocks (BSFA
-//               Figure 2b); gathers V rows of vertical columns
+//   warp 2      producer for V tiles; gathers V rows of vertical columns
 //   warp 3      idle
 //   warps 4-7   softmax warpgroup of Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup of Q tile 1
@@ -17,9 +15,9 @@
 // loaded once for all of them); without GQA they are four consecutive
 // q-blocks of one head.  Segments 0,1 form M = 128 tile 0 and segments 2,3
 // tile 1.  Each segment has a set of 64-key blocks (from the block table, the
-// causal range, the gate candidates or the vertical/slash lists); the unit
-// walks the 128-key tiles that hold a block of any segment, in ascending
-// order, and for each tile t with an active segment runs
+// causal range, the gate or the vertical/slash lists); the unit walks the
+// 128-key tiles that hold a block of any segment, in ascending order, and for
+// each tile t with an active segment runs
 //   S_t = Q_t K^T        tcgen05.mma M128 N128 K16 x 8, fp32 in TMEM
 //   softmax rows; P_t (bf16) written back over S_t in TMEM
 //   O_t += P_t V         tcgen05.mma with A from TMEM, M128 N128 K16 x 8
@@ -31,8 +29,22 @@
 // lse exact.  MMAs of one thread execute in issue order, so the commit that
 // signals S_t(e) also proves that PV_t(e-1) has read P_t(e-1) and written O_t.
 //
+// Gated mode (Block Sparse Flash Attention, Figure 2) runs each unit in two
+// phases.  Phase A, the gate, walks every causal key tile once and computes
+// S^T = K Q^T for both Q tiles in one M128 N256 MMA (keys on the TMEM lanes,
+// the 256 query rows on the columns; two such buffers fill all of TMEM, so
+// the next tile's product overlaps the reading of this one).  Each softmax
+// warp reads the 32 keys on its lanes and the 128 rows of its Q tile, takes
+// the maximum of each 32-key x 64-row piece, and compares it with the
+// segment's threshold: a 64 x 64 block's maximum is >= T exactly when the
+// maximum of one of its two 32-key pieces is, so each warp ORs its keep bit
+// into the unit's keep bitmap on its own (the diagonal block is always kept).
+// Phase B is block-table attention over the keep bitmaps: a pruned block
+// loads no V and runs no PV, and its keys are never exponentiated.
+//
 // TMEM (512 columns): tile t uses [256t, 256t+128) for S (fp32) / P (bf16
-// pairs, first 64 columns) and [256t+128, 256t+256) for O.
+// pairs, first 64 columns) and [256t+128, 256t+256) for O; the gate's two
+// S^T buffers are [0, 256) and [256, 512).
 #pragma once
 
 #include "sbfa_ptx.cuh"
@@ -46,7 +58,6 @@ constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kMaxKT = 8192;               // 64-key blocks: Sk <= 524288
 constexpr int kBmWords = kMaxKT / 32;
-constexpr int kDecRingSlots = 4;
 constexpr int kMaxCols = 1024;             // union of vertical columns per unit
 constexpr int kTileBytes = 64 * 128 * 2;   // 64 keys x 128 dims bf16
 constexpr int kKVTileBytes = 128 * 128 * 2;  // 128 keys: [d-chunk][128 rows][128 B]
@@ -90,7 +101,9 @@ struct PrefillParams {
 };
 
 struct PfSched {
-  uint32_t bm[4][kBmWords];
+  uint32_t bm[4][kBmWords];  // per segment: 64-key blocks to visit (gated: gate candidates)
+  // vertical-slash mode: the unit's column list; gated mode: the same words
+  // hold the keep bitmaps the gate writes ([4][kBmWords], see pf_kb)
   int col[kMaxCols];
   uint8_t colmask[kMaxCols];
   int n_words, n_cols;
@@ -98,14 +111,26 @@ struct PfSched {
   int seg_valid[4], seg_head[4], seg_row0[4], seg_qb[4];
   float seg_T[4];
 };
+static_assert(kMaxCols >= 4 * kBmWords, "keep bitmaps share the column list's storage");
+
+__device__ __forceinline__ uint32_t* pf_kb(PfSched& sc) {
+  return reinterpret_cast<uint32_t*>(sc.col);
+}
+
+// Pairing slot of the gate's exact block maximum: the two warps that hold
+// the two 32-key pieces of a 64-key half meet here (no waiting: the second
+// to arrive combines and writes).
+struct PfPair {
+  float v[2][2];  // [warp of the pair][segment of the tile]
+  int cnt;
+};
 
 struct PfSmem {
-  alignas(1024) uint8_t q[2][kQTileBytes];
+  alignas(1024) uint8_t q[2 * kQTileBytes];  // [64-dim chunk][tile][128 rows][128 B]
   alignas(1024) uint8_t k[kKStages][kKVTileBytes];
   alignas(1024) uint8_t v[kVStages][kKVTileBytes];
   PfSched sched[2];
-  float red[2][2][4][2];      // [tile][parity][warp][half] block-max exchange
-  int dec_val[kDecRingSlots][2];
+  PfPair pair[2][2][4];  // gate: [tile][key half][ring of items]
   int pv_flag[2];
   uint32_t tmem_base;
   int abort_flag;
@@ -114,32 +139,33 @@ struct PfSmem {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
-  uint64_t dec_full[kDecRingSlots], dec_empty[kDecRingSlots];
+  uint64_t ga_full[2], ga_free[2];  // gate: S^T buffers written / read
+  uint64_t kb_done;                 // gate: the unit's keep bitmaps are complete
   uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
 };
 
 static_assert(sizeof(PfSmem) + 1024 <= 232448, "prefill shared memory exceeds 227 KB");
 
-// Visit the 128-key tiles that hold a 64-key block of any segment (ascending),
-// then the vertical-column chunks of 128.  fn(kt, is_col, mem) where bit
-// (2s + h) of mem says segment s takes part in half h; stops when fn
-// returns false.
+// Visit the 128-key tiles that hold a 64-key block of any segment (ascending)
+// in the bitmaps `bits` ([4][kBmWords]), then the vertical-column chunks of
+// 128.  fn(kt, is_col, mem) where bit (2s + h) of mem says segment s takes
+// part in half h; stops when fn returns false.
 template <bool COLS, class F>
-__device__ __forceinline__ bool pf_for_each(const PfSched& sc, F&& fn) {
+__device__ __forceinline__ bool pf_for_each(const PfSched& sc, const uint32_t* bits, F&& fn) {
   for (int w = 0; w < sc.n_words; ++w) {
-    uint32_t bits[4];
+    uint32_t wb[4];
     uint32_t any = 0;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      bits[s] = sc.bm[s][w];
-      any |= (bits[s] | (bits[s] >> 1)) & 0x55555555u;
+      wb[s] = bits[s * kBmWords + w];
+      any |= (wb[s] | (wb[s] >> 1)) & 0x55555555u;
     }
     while (any) {
       const int bit = __ffs(any) - 1;  // even: half 0 of tile (32w + bit) / 2
       any &= any - 1u;
       int mem = 0;
 #pragma unroll
-      for (int s = 0; s < 4; ++s) mem |= ((bits[s] >> bit) & 3) << (2 * s);
+      for (int s = 0; s < 4; ++s) mem |= ((wb[s] >> bit) & 3) << (2 * s);
       if (!fn((w * 32 + bit) >> 1, false, mem)) return false;
     }
   }
@@ -173,6 +199,8 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
   const int g = bg % p.Hkv, b = bg / p.Hkv;
   const int n_words = (p.n_kt + 31) >> 5;
   for (int e = lane; e < 4 * kBmWords; e += 32) (&sc.bm[0][0])[e] = 0u;
+  if (p.mode == kModeGated)
+    for (int e = lane; e < 4 * kBmWords; e += 32) pf_kb(sc)[e] = 0u;
   if (lane == 0) {
     sc.n_words = n_words;
     sc.n_cols = 0;
@@ -294,6 +322,13 @@ __device__ __forceinline__ int pf_tile_halves(int mem, int t) {
   return (m | (m >> 2)) & 3;
 }
 
+// Byte offset of 64-dim chunk c of Q tile t (rows of both tiles are laid
+// out back to back within a chunk, so that the gate's N = 256 operand is one
+// K-major matrix).
+__device__ __forceinline__ uint32_t pf_q_off(int c, int t) {
+  return static_cast<uint32_t>(c * 2 * kQTileBytes / 2 + t * (kQTileBytes / 2));
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
@@ -318,6 +353,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.p_full[i], 128);
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.o_free[i], 128);
+      mbar_init(&sm.ga_full[i], 1);
+      mbar_init(&sm.ga_free[i], 8);  // one arrival per softmax warp
     }
     mbar_init(&sm.q_empty, 1);
     for (int i = 0; i < kKStages; ++i) {
@@ -328,11 +365,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
-    for (int i = 0; i < kDecRingSlots; ++i) {
-      mbar_init(&sm.dec_full[i], 2);
-      mbar_init(&sm.dec_empty[i], 1);
-    }
+    mbar_init(&sm.kb_done, 8);
     mbar_init(&sm.mma_drain, 1);
+    for (int i = 0; i < 16; ++i) (&sm.pair[0][0][0])[i].cnt = 0;
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -389,7 +424,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               const int s = 2 * t + h;
               if (!sc.seg_valid[s]) continue;
               for (int c = 0; c < 2; ++c)
-                tma_load_4d(sm.q[t] + c * 16384 + h * 8192, &mapQ, &sm.q_full[t], c * 64,
+                tma_load_4d(sm.q + pf_q_off(c, t) + h * 8192, &mapQ, &sm.q_full[t], c * 64,
                             sc.seg_head[s], sc.seg_row0[s], sc.b);
             }
           }
@@ -424,7 +459,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (++ks == kKStages) { ks = 0; kph ^= 1u; }
         return true;
       };
-      ok = pf_for_each<has_cols>(sc, body);
+      if (gated) {
+        // phase A (the gate) over the candidates, then phase B over what it kept
+        ok = pf_for_each<false>(sc, &sc.bm[0][0], body);
+        if (ok && lane == 0) ok = mbar_wait(&sm.kb_done, n & 1, wctx);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (ok) ok = pf_for_each<false>(sc, pf_kb(sc), body);
+      } else {
+        ok = pf_for_each<has_cols>(sc, &sc.bm[0][0], body);
+      }
     }
     // no copy may still be landing in shared memory when the CTA exits
     if (lane == 0) {
@@ -438,32 +481,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int vs = 0;
     uint32_t vph = 0;
     uint32_t v_armed = 0, v_par = 0;  // as k_armed / k_par above
-    int dslot = 0;
-    uint32_t dph = 0;
     bool ok = true;
     int n = 0;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
       const int ub = n & 1;
       PfSched& sc = sm.sched[ub];
-      if (lane == 0) ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
+      if (lane == 0) {
+        ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
+        if (gated && ok) ok = mbar_wait(&sm.kb_done, n & 1, wctx);
+      }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       auto body = [&](int kt, bool is_col, int mem) -> bool {
         bool good = true;
-        int need = (mem | (mem >> 2) | (mem >> 4) | (mem >> 6)) & 3;
-        if (gated) {
-          if (lane == 0) {
-            good = mbar_wait_t(&sm.dec_full[dslot], dph, wctx, pacc[1]);
-            if (good) {
-              need = sm.dec_val[dslot][0] | sm.dec_val[dslot][1];
-              mbar_arrive(&sm.dec_empty[dslot]);
-            }
-          }
-          if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
-          good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
-          need = __shfl_sync(0xffffffffu, need, 0);
-          if (!good) return false;
-        }
+        const int need = (mem | (mem >> 2) | (mem >> 4) | (mem >> 6)) & 3;
         if (!need) return true;
         if (lane == 0) good = mbar_wait_t(&sm.v_empty[vs], vph ^ 1u, wctx, pacc[0]);
         good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
@@ -489,7 +520,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (++vs == kVStages) { vs = 0; vph ^= 1u; }
         return true;
       };
-      ok = pf_for_each<has_cols>(sc, body);
+      ok = pf_for_each<has_cols>(sc, gated ? pf_kb(sc) : &sc.bm[0][0], body);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sched_empty[ub]);
     }
@@ -501,18 +532,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 128, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
-      // base descriptors; K-step and stage offsets are added to the start
-      // address field (bits 0-13, 16-byte units), which cannot overflow inside
-      // the shared window
-      const uint64_t qdesc0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      const uint32_t idesc_ga = idesc_bf16(128, 256, 0);
+      // base descriptors; K-step, tile and stage offsets are added to the
+      // start address field (bits 0-13, 16-byte units), which cannot overflow
+      // inside the shared window
+      const uint64_t qdesc0 = sdesc_sw128(smem_u32(sm.q), 16, 1024);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.v[0]), 16384, 1024);
       int ks = 0, vs = 0;
       uint32_t kph = 0, vph = 0;
       uint32_t pph = 0;   // bit t: p_full[t] phase
       uint32_t ofph = 0;  // bit t: o_free[t] phase
+      int ai = 0;         // gate items issued so far (S^T buffer ai & 1)
       bool ok = true;
       int n = 0;
+      // start-address offsets of K-step kk: Q (chunk stride 2 tiles) and K
+      auto q_step = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 2 * kQTileBytes / 2 + (kk & 3) * 32) >> 4); };
+      auto k_step = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
         const int ub = n & 1;
         PfSched& sc = sm.sched[ub];
@@ -523,6 +559,39 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!ok) break;
         int pv_started = 0;    // bit t
         int ofree_waited = 0;  // bit t
+        if (gated) {
+          // The gate's S^T buffers cover all of TMEM, O included: the previous
+          // unit's epilogue must have read O first.
+          for (int t = 0; t < 2 && ok; ++t) {
+            ok = mbar_wait_t(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx, pacc[4]);
+            ofph ^= 1u << t;
+          }
+          ofree_waited = 3;
+          if (!ok) break;
+          tc_fence_after();
+          auto gate = [&](int kt, bool, int) -> bool {
+            if (!mbar_wait_t(&sm.k_full[ks], kph, wctx, pacc[0])) return false;
+            const int b = ai & 1;
+            if (!mbar_wait_t(&sm.ga_free[b], ((ai >> 1) & 1) ^ 1u, wctx, pacc[2])) return false;
+            tc_fence_after();
+            const uint64_t kd = kdesc0 + static_cast<uint64_t>((ks * kKVTileBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ss(tmem + b * 256, kd + k_step(kk), qdesc0 + q_step(kk), idesc_ga, kk ? 1u : 0u);
+            umma_commit(&sm.ga_full[b]);
+            umma_commit(&sm.k_empty[ks]);
+            if (++ks == kKStages) { ks = 0; kph ^= 1u; }
+            ++ai;
+            return true;
+          };
+          ok = pf_for_each<false>(sc, &sc.bm[0][0], gate);
+          // phase B reuses the S^T buffers: both must have been read
+          for (int i = 1; i <= 2 && ok && ai - i >= 0; ++i)
+            ok = mbar_wait_t(&sm.ga_free[(ai - i) & 1], ((ai - i) >> 1) & 1, wctx, pacc[2]);
+          if (ok) ok = mbar_wait(&sm.kb_done, n & 1, wctx);
+          if (!ok) break;
+          tc_fence_after();
+        }
         // Issue order (two-tile ping-pong): QK(e,t0), PV(e-1,t1), QK(e,t1),
         // PV(e,t0).  Each softmax warpgroup then computes while the tensor core
         // runs the other tile's work.  The V stage of item e is released after
@@ -572,12 +641,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           return true;
         };
         auto issue_qk = [&](int t, uint64_t kd) {
-          const uint64_t qd = qdesc0 + static_cast<uint64_t>((t * kQTileBytes) >> 4);
+          const uint64_t qd = qdesc0 + static_cast<uint64_t>(pf_q_off(0, t) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-            umma_ss(tmem + t * 256, qd + off, kd + off, idesc_qk, kk ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + t * 256, qd + q_step(kk), kd + k_step(kk), idesc_qk, kk ? 1u : 0u);
           umma_commit(&sm.s_full[t]);
         };
         auto body = [&](int kt, bool is_col, int mem) -> bool {
@@ -606,7 +673,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           pend = {1, (act >> 1) & 1, f0, v_waited};
           return true;
         };
-        ok = pf_for_each<has_cols>(sc, body);
+        ok = pf_for_each<has_cols>(sc, gated ? pf_kb(sc) : &sc.bm[0][0], body);
         if (ok && pend.valid) ok = finish_prev();
         for (int t = 0; t < 2 && ok; ++t) {
           if (!((ofree_waited >> t) & 1)) {
@@ -630,24 +697,104 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int quarter = (warp & 3);
     const int hseg = r >> 6;              // 0/1: segment within tile
     const int seg = 2 * t + hseg;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 256;
-    const int bar_id = 1 + t;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t lane_addr = lane_base + t * 256;
     const float NEG = -INFINITY;
     uint32_t sph = 0;
-    int dslot = 0;
-    uint32_t dph = 0;
-    int dbuf = 0;
     uint32_t pv_total = 0;  // PVs issued for this tile so far (pv_done phases)
+    int ai = 0;             // gate items read so far
     bool ok = true;
     int n = 0;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n) {
       const int ub = n & 1;
       PfSched& sc = sm.sched[ub];
-      ok = mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx);
-      // gated mode synchronises the warpgroup on named barriers: its four
-      // warps must leave together, so every exit is agreed on one first
-      if (gated) ok = !named_bar_or(bar_id, 128, !ok);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.sched_full[ub], (n >> 1) & 1, wctx));
       if (!ok) break;
+      if (gated) {
+        // ---- phase A: the gate.  This warp holds keys 32*quarter .. +31 of
+        // each tile (lanes) and the 128 rows of Q tile t (columns).
+        const int key_l = quarter * 32 + lane;
+        const int h = quarter >> 1;
+        auto gate = [&](int kt, bool, int mem) -> bool {
+          const int b = ai & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait_t(&sm.ga_full[b], (ai >> 1) & 1, wctx, pacc[0])))
+            return false;
+          tc_fence_after();
+          const int key = kt * 128 + key_l;
+          const int j = 2 * kt + h;  // 64-key block of this warp's keys
+          float wm[2];
+#pragma unroll
+          for (int ss = 0; ss < 2; ++ss) {
+            const int s = 2 * t + ss;
+            const int row0 = sc.seg_row0[s];
+            // visible query rows row0 + c of this key: c in [lo, hi)
+            int lo = 0, hi = min(64, p.Sq - row0);
+            if (p.causal) lo = max(0, key - row0 - p.causal_off);
+            if (!((mem >> (2 * s + h)) & 1) || key >= p.Sk) hi = 0;
+            float x[64];
+            tmem_ld64(lane_base + b * 256 + t * 128 + ss * 64, x);
+            float m4[4] = {NEG, NEG, NEG, NEG};
+            if (lo == 0 && hi == 64) {
+#pragma unroll
+              for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], x[c], x[c + 1]);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 64; ++c)
+                m4[c & 3] = fmaxf(m4[c & 3], (c >= lo && c < hi) ? x[c] : NEG);
+            }
+            wm[ss] = warp_max_f32(fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sm.ga_free[b]);
+            uint32_t* kb = pf_kb(sc);
+#pragma unroll
+            for (int ss = 0; ss < 2; ++ss) {
+              const int s = 2 * t + ss;
+              if (!((mem >> (2 * s + h)) & 1)) continue;
+              // BSFA Figure 2b: keep iff diagonal or s_max >= T
+              if (j == sc.seg_qb[s] || wm[ss] * p.scale >= sc.seg_T[s])
+                atomicOr(&kb[s * kBmWords + (j >> 5)], 1u << (j & 31));
+            }
+            if (p.smax_out) {
+              // exact block maximum: the two warps of this key half pair up
+              PfPair& ps = sm.pair[t][h][ai & 3];
+              ps.v[quarter & 1][0] = wm[0];
+              ps.v[quarter & 1][1] = wm[1];
+              __threadfence_block();
+              if (atomicAdd(&ps.cnt, 1) == 1) {
+                __threadfence_block();
+#pragma unroll
+                for (int ss = 0; ss < 2; ++ss) {
+                  const int s = 2 * t + ss;
+                  if (!((mem >> (2 * s + h)) & 1)) continue;
+                  const float bm = fmaxf(wm[ss], ps.v[(quarter & 1) ^ 1][ss]);
+                  p.smax_out[((static_cast<int64_t>(sc.b) * p.Hq + sc.seg_head[s]) * p.nqb +
+                              sc.seg_qb[s]) * p.nqb + j] = bm * p.scale;
+                }
+                ps.cnt = 0;
+              }
+            }
+          }
+          ++ai;
+          return true;
+        };
+        ok = pf_for_each<false>(sc, &sc.bm[0][0], gate);
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.kb_done);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.kb_done, n & 1, wctx));
+        if (!ok) break;
+        if (p.keep_out && sc.seg_valid[seg]) {
+          const uint32_t* kb = pf_kb(sc) + seg * kBmWords;
+          const int qb = sc.seg_qb[seg];
+          uint8_t* dst = p.keep_out + ((static_cast<int64_t>(sc.b) * p.Hq + sc.seg_head[seg]) * p.nqb +
+                                       qb) * p.nqb;
+          for (int jj = (r & 63); jj <= qb; jj += 64) dst[jj] = (kb[jj >> 5] >> (jj & 31)) & 1u;
+        }
+      }
+      // ---- attention over the unit's blocks (gated: the blocks the gate kept)
       const int my_valid = sc.seg_valid[seg];
       const int my_row = sc.seg_row0[seg] + (r & 63);
       const bool row_ok = my_valid && my_row < p.Sq;
@@ -655,26 +802,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int npv = 0;
       auto body = [&](int kt, bool is_col, int mem) -> bool {
         const int tmask = pf_tile_halves(mem, t);
-        if (!tmask) {
-          if (gated) {
-            bool fail = false;
-            if (r == 0) fail = !mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2]);
-            // every wait result is agreed on before anyone leaves: the named
-            // barriers below must always see all 128 threads
-            if (named_bar_or(bar_id, 128, fail)) return false;
-            if (r == 0) {
-              sm.dec_val[dslot][t] = 0;
-              mbar_arrive(&sm.dec_full[dslot]);
-            }
-            if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
-          }
-          return true;
-        }
+        if (!tmask) return true;
         const int segm = row_ok ? (mem >> (2 * seg)) & 3 : 0;
-        bool okw = mbar_wait_t(&sm.s_full[t], sph, wctx, pacc[0]);
         // tcgen05.ld below is warp-collective: the warp leaves together
-        okw = __all_sync(0xffffffffu, okw);
-        if (!gated && !okw) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait_t(&sm.s_full[t], sph, wctx, pacc[0]))) return false;
         sph ^= 1u;
         tc_fence_after();
         pacc[5] += 1;
@@ -700,64 +831,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         };
         float rm[2] = {NEG, NEG};
-        if (okw) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float sh[64];
-            tmem_ld64(lane_addr + 64 * h, sh);
-            mask_half(sh, h);
-            float m4[4] = {NEG, NEG, NEG, NEG};
+        for (int h = 0; h < 2; ++h) {
+          float sh[64];
+          tmem_ld64(lane_addr + 64 * h, sh);
+          mask_half(sh, h);
+          float m4[4] = {NEG, NEG, NEG, NEG};
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], sh[c], sh[c + 1]);
-            rm[h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          }
+          for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], sh[c], sh[c + 1]);
+          rm[h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
-        int my_keep = segm;
-        int flag = tmask;
-        if (gated) {
-          // exact block max of each 64 x 64 sub-tile (BSFA Figure 2a)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const float wm = warp_max_f32(rm[h]);
-            if (lane == 0) sm.red[t][dbuf][quarter][h] = wm;
-          }
-          bool fail = !okw;
-          if (r == 0 && !fail) fail = !mbar_wait_t(&sm.dec_empty[dslot], dph ^ 1u, wctx, pacc[2]);
-          if (named_bar_or(bar_id, 128, fail)) return false;
-          flag = 0;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int sgi = 2 * t + hh;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const bool act = (mem >> (2 * sgi + h)) & 1;
-              const float bmax = fmaxf(sm.red[t][dbuf][2 * hh][h], sm.red[t][dbuf][2 * hh + 1][h]);
-              const float smax = bmax * p.scale;
-              const int j = 2 * kt + h;
-              const bool keep = act && (j == sc.seg_qb[sgi] || smax >= sc.seg_T[sgi]);
-              if (keep) flag |= 1 << h;
-              if (hh == hseg) my_keep = (my_keep & ~(1 << h)) | ((keep && row_ok) ? 1 << h : 0);
-              if (act && r == 64 * hh + h) {
-                const int64_t oi =
-                    ((static_cast<int64_t>(sc.b) * p.Hq + sc.seg_head[sgi]) * p.nqb +
-                     sc.seg_qb[sgi]) * p.nqb + j;
-                if (p.smax_out) p.smax_out[oi] = smax;
-                if (p.keep_out) p.keep_out[oi] = keep ? 1 : 0;
-              }
-            }
-          }
-          dbuf ^= 1;
-          if (r == 0) {
-            sm.dec_val[dslot][t] = flag;
-            mbar_arrive(&sm.dec_full[dslot]);
-          }
-          if (++dslot == kDecRingSlots) { dslot = 0; dph ^= 1u; }
-        }
-        if (!flag) {
-          if (r == 0) sm.pv_flag[t] = 0;
-          mbar_arrive(&sm.p_full[t]);
-          return true;
-        }
+        const int my_keep = segm;
+        const int flag = tmask;
         // ---- online softmax over the kept halves (log2 domain, lazy rescale)
         float rmax = NEG;
         if (my_keep & 1) rmax = rm[0];
@@ -826,16 +911,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         pacc[7] += 1;
         return true;
       };
-      ok = pf_for_each<has_cols>(sc, body);
+      ok = pf_for_each<has_cols>(sc, gated ? pf_kb(sc) : &sc.bm[0][0], body);
       if (!ok) break;
       // ---- epilogue: o = O / l, lse = ln(sum)
       const bool store = row_ok;
       const int head = sc.seg_head[seg];
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       if (npv > 0) {
-        bool okd = __all_sync(0xffffffffu,
-                              mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1]));
-        if (gated) okd = !named_bar_or(bar_id, 128, !okd);  // npv is uniform in the warpgroup
+        const bool okd = __all_sync(0xffffffffu,
+                                    mbar_wait_t(&sm.pv_done[t], (pv_total - 1) & 1, wctx, pacc[1]));
         if (!okd) { ok = false; break; }
         tc_fence_after();
         float ob[32];

@@ -264,7 +264,8 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
                           const sbfa_t4* kA, const sbfa_t4* vA, int S_A, int causal_A,
                           const sbfa_t4* kB, const sbfa_t4* vB, const sbfa_table* tb, void* ws,
                           size_t ws_bytes, const sbfa_t4& o, float* lse, int32_t* status,
-                          cudaStream_t stream, int grid_cap = 0, int ticket_pairs = 0) {
+                          cudaStream_t stream, int grid_cap = 0, int ticket_pairs = 0,
+                          bool dedup = false) {
   DevInfo di;
   SBFA_TRY(dev_info(&di));
   const int G = s->Hq / s->Hkv;
@@ -329,11 +330,16 @@ sbfa_status launch_decode(sbfa::DecodeParams& p, const sbfa_shape* s, const sbfa
   int dev = 0;
   SBFA_CUDA(cudaGetDevice(&dev));
   if (!attr_set[dev]) {
-    SBFA_CUDA(cudaFuncSetAttribute(sbfa::decode_kernel,
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::decode_kernel<false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::decode_kernel<true>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr_set[dev] = true;
   }
-  sbfa::decode_kernel<<<grid, sbfa::kDecThreads, smem, stream>>>(p);
+  if (dedup)
+    sbfa::decode_kernel<true><<<grid, sbfa::kDecThreads, smem, stream>>>(p);
+  else
+    sbfa::decode_kernel<false><<<grid, sbfa::kDecThreads, smem, stream>>>(p);
   SBFA_CUDA(cudaGetLastError());
   return SBFA_OK;
 }
@@ -469,9 +475,9 @@ sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
   SBFA_TRY(check_table(table, shape, !dec));
   if (dec) {
     sbfa::DecodeParams p{};
-    p.dedup = 1;  // a row is a set of blocks, as on the tiled kernel
+    // a row is a set of blocks, as on the tiled kernel
     return launch_decode(p, shape, q, nullptr, nullptr, 0, 0, &k, &v, table, nullptr, 0, o,
-                         lse, status, reinterpret_cast<cudaStream_t>(stream));
+                         lse, status, reinterpret_cast<cudaStream_t>(stream), 0, 0, true);
   }
   sbfa::PrefillParams p{};
   p.mode = sbfa::kModeTable;
