@@ -545,8 +545,8 @@ def oracle_sample_vs_convert(wl, n_qb=32):
     oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True, qblocks=qbs)
     sec = time.perf_counter() - t0
     return {"kind": "oracle", "unit": "s", "cores": os.cpu_count(),
-            "sample": f"conversion of {n_qb} q-blocks of head 0", "sample_seconds": round(sec, 3),
-            "extrapolated_full_seconds": round(sec * nqb * H / n_qb, 3)}
+            "sample": f"conversion of {n_qb} q-blocks of head 0", "sample_seconds": round(sec, 6),
+            "extrapolated_full_seconds": round(sec * nqb * H / n_qb, 6)}
 
 
 def nsa_sample_pairs(cu, sel, toks):

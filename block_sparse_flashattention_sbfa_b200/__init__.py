@@ -62,6 +62,13 @@ _SIGS = {
                                     _P, _P, _P],
     "sbfa_fwd_vertical_slash": [ctypes.POINTER(Shape), T4, T4, T4, _P, _P, _I, _P, _P, _I, _I,
                                 _I, T4, _P, _P, _P],
+    "sbfa_convert_vertical_slash_mergehead": [_P, _P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _I, _I,
+                                              _I, _P, _P, _P, _P, _P, _P],
+    "sbfa_fwd_varlen": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, T4, T4, T4,
+                        ctypes.POINTER(Table), T4, _P, _P, _P],
+    "sbfa_fwd_vertical_slash_varlen": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                                       _I, T4, T4, T4, _P, _P, _I, _P, _P, _I, _I, _I, T4, _P,
+                                       _P, _P],
     "sbfa_fwd_varlen_selected": [_P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, T4, T4, T4, _P,
                                  _I, _I, _P, ctypes.c_size_t, T4, _P, _P, _P],
     "sbfa_varlen_selected_workspace_size": [_I, _I, _I, _I, _I, _I],
@@ -283,6 +290,83 @@ def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
           block_N, int(bool(causal)), bc.data_ptr(), bo.data_ptr(), cc.data_ptr(),
           ci.data_ptr(), _ptr(status), _stream())
     return bc, bo, cc, ci
+
+
+def convert_vertical_slash_mergehead(q_seqlens, kv_seqlens, vertical, slash, vertical_count,
+                                     slash_count, context_size, block_M=64, block_N=64,
+                                     causal=True, status=None):
+    """``sbfa_convert_vertical_slash_mergehead``: as convert_vertical_slash,
+    with head h using only the first vertical_count[h] / slash_count[h]
+    entries of its rows (int32 (H,) device tensors)."""
+    B, H, nnz_v = vertical.shape
+    nnz_s = slash.shape[2]
+    nqb = -(-context_size // block_M)
+    dev = vertical.device
+    for t in (q_seqlens, kv_seqlens, vertical, slash, vertical_count, slash_count):
+        if t.dtype != torch.int32 or not t.is_contiguous():
+            raise TypeError("index inputs must be contiguous int32")
+    bc = torch.empty(B, H, nqb, dtype=torch.int32, device=dev)
+    bo = torch.empty(B, H, nqb, nnz_s, dtype=torch.int32, device=dev)
+    cc = torch.empty(B, H, nqb, dtype=torch.int32, device=dev)
+    ci = torch.empty(B, H, nqb, nnz_v, dtype=torch.int32, device=dev)
+    _call("sbfa_convert_vertical_slash_mergehead", q_seqlens.data_ptr(), kv_seqlens.data_ptr(),
+          vertical.data_ptr(), nnz_v, slash.data_ptr(), nnz_s, vertical_count.data_ptr(),
+          slash_count.data_ptr(), B, H, context_size, block_M, block_N, int(bool(causal)),
+          bc.data_ptr(), bo.data_ptr(), cc.data_ptr(), ci.data_ptr(), _ptr(status), _stream())
+    return bc, bo, cc, ci
+
+
+def _varlen_args(q, k, cu_seqlens_q, cu_seqlens_k):
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("cu_seqlens must be contiguous int32 CUDA tensors")
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("varlen q, k, v are (total, heads, dim)")
+    return cu_seqlens_q.numel() - 1, q.shape[0], k.shape[0]
+
+
+def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, table, q_block,
+               kv_block, causal=False, scale=None, out=None, lse=None, status=None):
+    """Block-table attention over cu_seqlens-packed sequences
+    (``sbfa_fwd_varlen``).  q (total_q, Hq, D), k/v (total_k, Hkv, D), table
+    int32 (nseq, Hkv, nQB, nmax) of sequence-local blocks.  Returns
+    o (total_q, Hq, D), lse (Hq, total_q)."""
+    _check_bf16(q, k, v)
+    nseq, tq, tk = _varlen_args(q, k, cu_seqlens_q, cu_seqlens_k)
+    Hq, D = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, tq, dtype=torch.float32, device=q.device)
+    tb = _table(table, q_block, kv_block)
+    _call("sbfa_fwd_varlen", cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), nseq, tq, tk,
+          int(max_seqlen_q), int(max_seqlen_k), Hq, k.shape[1], D,
+          0.0 if scale is None else float(scale), int(bool(causal)), _t4(q[None]), _t4(k[None]),
+          _t4(v[None]), ctypes.byref(tb), _t4(out[None]), lse.data_ptr(), _ptr(status), _stream())
+    return out, lse
+
+
+def fwd_vertical_slash_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                              block_count, block_offset, column_count, column_index, causal=True,
+                              scale=None, block_M=64, block_N=64, out=None, lse=None,
+                              status=None):
+    """``sbfa_fwd_vertical_slash_varlen``: vertical/slash attention over
+    cu_seqlens-packed sequences; index arrays (nseq, Hq, ceil(max_seqlen_q /
+    64), nnz).  Returns o (total_q, Hq, D), lse (Hq, total_q)."""
+    _check_bf16(q, k, v)
+    nseq, tq, tk = _varlen_args(q, k, cu_seqlens_q, cu_seqlens_k)
+    Hq, D = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, tq, dtype=torch.float32, device=q.device)
+    _call("sbfa_fwd_vertical_slash_varlen", cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+          nseq, tq, tk, int(max_seqlen_q), int(max_seqlen_k), Hq, k.shape[1], D,
+          0.0 if scale is None else float(scale), int(bool(causal)), _t4(q[None]), _t4(k[None]),
+          _t4(v[None]), block_count.data_ptr(), block_offset.data_ptr(), block_offset.shape[-1],
+          column_count.data_ptr(), column_index.data_ptr(), column_index.shape[-1], block_M,
+          block_N, _t4(out[None]), lse.data_ptr(), _ptr(status), _stream())
+    return out, lse
 
 
 def calibrate_thresholds(smax, k_top, T=None):

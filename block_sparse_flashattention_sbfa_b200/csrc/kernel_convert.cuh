@@ -1,5 +1,8 @@
 // Vertical/slash index conversion (Sglang Sparse Flash Attention,
-// convert_vertical_slash_indexes): one CTA per (batch, head, q-block).
+// convert_vertical_slash_indexes, and the per-head-count variant
+// convert_vertical_slash_indexes_mergehead): one CTA per (batch, head,
+// q-block).  With per-head counts, head h uses only the first v_cnt[h]
+// vertical and s_cnt[h] slash entries of its rows.
 //
 // Slash offset s is the diagonal key = row + d - s (d = kv_len - q_len); over
 // the q-block's rows [m0, m1) it covers keys [m0+d-s, m1-1+d-s].  Each such
@@ -39,7 +42,8 @@ __device__ __forceinline__ int cv_block_scan(int v, int* warp_tot, int& excl) {
 __global__ void __launch_bounds__(kCvThreads)
     convert_vs_kernel(const int* __restrict__ q_seqlens, const int* __restrict__ kv_seqlens,
                       const int* __restrict__ vertical, int nnz_v, const int* __restrict__ slash,
-                      int nnz_s, int H, int nqb, int block_M, int block_N, int causal,
+                      int nnz_s, const int* __restrict__ v_cnt, const int* __restrict__ s_cnt,
+                      int H, int nqb, int block_M, int block_N, int causal,
                       int* __restrict__ block_count, int* __restrict__ block_offset,
                       int* __restrict__ column_count, int* __restrict__ column_index,
                       int* status) {
@@ -50,6 +54,10 @@ __global__ void __launch_bounds__(kCvThreads)
   const int b = bh / H;
   const int tid = threadIdx.x;
   const int q_len = q_seqlens[b], kv_len = kv_seqlens[b];
+  // entries of this head's rows in use (the row strides stay nnz_v / nnz_s)
+  const int h = bh % H;
+  const int nv = v_cnt ? min(max(v_cnt[h], 0), nnz_v) : nnz_v;
+  const int ns = s_cnt ? min(max(s_cnt[h], 0), nnz_s) : nnz_s;
   const int d = kv_len - q_len;
   const int64_t row = static_cast<int64_t>(bh) * nqb + i;
   const int m0 = i * block_M;
@@ -66,7 +74,7 @@ __global__ void __launch_bounds__(kCvThreads)
   for (int w = tid; w < nwords; w += kCvThreads) bm[w] = 0u;
   __syncthreads();
   const int* sl = slash + static_cast<int64_t>(bh) * nnz_s;
-  for (int e = tid; e < nnz_s; e += kCvThreads) {
+  for (int e = tid; e < ns; e += kCvThreads) {
     const int s = sl[e];
     if (s < 0) { report(status, kDevBadIndex); continue; }
     const int lo = max(m0 + d - s, 0);
@@ -102,11 +110,11 @@ __global__ void __launch_bounds__(kCvThreads)
   int* ci = column_index + row * nnz_v;
   const int vis_end = causal ? min(kv_len, m1 + d) : kv_len;  // columns < vis_end
   int ncol = 0;
-  for (int e0 = 0; e0 < nnz_v; e0 += kCvThreads) {
+  for (int e0 = 0; e0 < nv; e0 += kCvThreads) {
     const int e = e0 + tid;
     int c = -1;
     bool keep = false;
-    if (e < nnz_v) {
+    if (e < nv) {
       c = vt[e];
       keep = c >= 0 && c < vis_end && !((bm[(c / block_N) >> 5] >> ((c / block_N) & 31)) & 1u);
       if (c < 0) report(status, kDevBadIndex);

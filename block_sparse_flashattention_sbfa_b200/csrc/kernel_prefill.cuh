@@ -74,6 +74,12 @@ struct PrefillParams {
   int64_t osb, oss, osh;
   int o_f32;
   float* lse;
+  int64_t lse_sb, lse_sh;  // lse element strides of batch (sequence) and head
+  // varlen: sequences packed along the row axis by cumulative lengths
+  // (nullptr: batched layout); the batch index is then the sequence index,
+  // Sq / Sk are the longest lengths and o / lse are indexed by packed row
+  const int* cu_q;
+  const int* cu_k;
   // table mode
   const int* idx;
   int64_t tsb, tsh, tsqb;
@@ -108,6 +114,9 @@ struct PfSched {
   uint8_t colmask[kMaxCols];
   int n_words, n_cols;
   int b, g;
+  int tb;                  // batch coordinate of the TMA maps (0 when varlen)
+  int q_base, q_len;       // the unit's query rows: packed offset and length
+  int k_base, k_len, coff;  // its keys; causal offset k_len - q_len
   int seg_valid[4], seg_head[4], seg_row0[4], seg_qb[4];
   float seg_T[4];
 };
@@ -139,6 +148,11 @@ struct PfSmem {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  // o_ack[t]: the MMA warp has taken note of tile t's previous o_free phase.
+  // A tile with no block in a unit finishes its epilogue at once; without
+  // this handshake its o_free could complete a second phase before the MMA
+  // warp waits for the first, and the parity test would then wait forever.
+  uint64_t o_ack[2];
   uint64_t ga_full[2], ga_free[2];  // gate: S^T buffers written / read
   uint64_t kb_done;                 // gate: the unit's keep bitmaps are complete
   uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
@@ -198,6 +212,17 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
   const int bg = rest / p.n_hgrp;
   const int g = bg % p.Hkv, b = bg / p.Hkv;
   const int n_words = (p.n_kt + 31) >> 5;
+  int q_base = 0, q_len = p.Sq, k_base = 0, k_len = p.Sk;
+  if (p.cu_q) {
+    q_base = __ldg(p.cu_q + b);
+    q_len = __ldg(p.cu_q + b + 1) - q_base;
+    k_base = __ldg(p.cu_k + b);
+    k_len = __ldg(p.cu_k + b + 1) - k_base;
+  }
+  const int coff = k_len - q_len;
+  const int n_sub = (q_len + 63) / 64;
+  const int n_kt = (k_len + 63) / 64;
+  const int n_kb = p.mode == kModeTable ? (k_len + p.kv_block - 1) / p.kv_block : 0;
   for (int e = lane; e < 4 * kBmWords; e += 32) (&sc.bm[0][0])[e] = 0u;
   if (p.mode == kModeGated)
     for (int e = lane; e < 4 * kBmWords; e += 32) pf_kb(sc)[e] = 0u;
@@ -206,13 +231,19 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
     sc.n_cols = 0;
     sc.b = b;
     sc.g = g;
+    sc.tb = p.cu_q ? 0 : b;
+    sc.q_base = q_base;
+    sc.q_len = q_len;
+    sc.k_base = k_base;
+    sc.k_len = k_len;
+    sc.coff = coff;
   }
   __syncwarp();
   for (int s = 0; s < 4; ++s) {
     const int hs = s % p.hp, ss = s / p.hp;
     const int head = g * p.G + hgrp * p.hp + hs;
     const int sub = sg * p.subs_per_unit + ss;
-    const int valid = sub < p.n_sub;
+    const int valid = sub < n_sub;
     const int row0 = sub * 64;
     if (lane == 0) {
       sc.seg_valid[s] = valid;
@@ -223,11 +254,11 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
     }
     if (!valid) continue;
     // causal limit: last tile any row of the segment may see
-    int kt_end = p.n_kt;
+    int kt_end = n_kt;
     if (p.causal) {
-      const int last_row = min(row0 + 63, p.Sq - 1);
-      const int max_key = last_row + p.causal_off;
-      kt_end = max_key < 0 ? 0 : min(p.n_kt, max_key / 64 + 1);
+      const int last_row = min(row0 + 63, q_len - 1);
+      const int max_key = last_row + coff;
+      kt_end = max_key < 0 ? 0 : min(n_kt, max_key / 64 + 1);
     }
     uint32_t* bm = sc.bm[s];
     if (p.mode == kModeDense || p.mode == kModeGated) {
@@ -242,7 +273,7 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
       for (int n = lane; n < p.nmax; n += 32) {
         const int j = row[n];
         if (j < 0) continue;
-        if (j >= p.n_kb) { report(p.status, kDevBadIndex); continue; }
+        if (j >= n_kb) { report(p.status, kDevBadIndex); continue; }
         pf_set_range(bm, j * tpb, min(kt_end, j * tpb + tpb));
       }
     } else {  // vertical-slash: listed blocks
@@ -251,7 +282,7 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
       const int* offs = p.vs_bo + base * p.nnz_s;
       for (int n = lane; n < cnt; n += 32) {
         const int off = offs[n];
-        if (off < 0 || off >= p.Sk || (off & 63)) { report(p.status, kDevBadIndex); continue; }
+        if (off < 0 || off >= k_len || (off & 63)) { report(p.status, kDevBadIndex); continue; }
         const int t = off >> 6;
         if (t < kt_end) atomicOr(&bm[t >> 5], 1u << (t & 31));
       }
@@ -281,7 +312,7 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
       int mem = 0;
       for (int s = 0; s < 4; ++s)
         if (cur[s] < cnt[s] && lst[s][cur[s]] == best) { mem |= 1 << s; ++cur[s]; }
-      if (best < 0 || best >= p.Sk) { report(p.status, kDevBadIndex); continue; }
+      if (best < 0 || best >= k_len) { report(p.status, kDevBadIndex); continue; }
       if (n == kMaxCols) { report(p.status, kDevOverflow); break; }
       sc.col[n] = best;
       sc.colmask[n] = static_cast<uint8_t>(mem);
@@ -304,8 +335,9 @@ __device__ __forceinline__ void pf_gather_rows(const PfSched& sc, int e0, int ha
     const uint32_t saddr = d0 + (ch >> 3) * 16384 + sw128_off(r, ch & 7);
     const int idx = e0 + r;
     if (idx < sc.n_cols) {
-      const __nv_bfloat16* src = base + sc.b * sb + static_cast<int64_t>(sc.col[idx]) * ss +
-                                 sc.g * sh + ch * 8;
+      const __nv_bfloat16* src = base + sc.tb * sb +
+                                 static_cast<int64_t>(sc.k_base + sc.col[idx]) * ss + sc.g * sh +
+                                 ch * 8;
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(src) : "memory");
     } else {
       asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(saddr), "r"(0) : "memory");
@@ -353,6 +385,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.p_full[i], 128);
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.o_free[i], 128);
+      mbar_init(&sm.o_ack[i], 1);
       mbar_init(&sm.ga_full[i], 1);
       mbar_init(&sm.ga_free[i], 8);  // one arrival per softmax warp
     }
@@ -425,7 +458,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!sc.seg_valid[s]) continue;
               for (int c = 0; c < 2; ++c)
                 tma_load_4d(sm.q + pf_q_off(c, t) + h * 8192, &mapQ, &sm.q_full[t], c * 64,
-                            sc.seg_head[s], sc.seg_row0[s], sc.b);
+                            sc.seg_head[s], sc.q_base + sc.seg_row0[s], sc.tb);
             }
           }
         }
@@ -447,7 +480,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!((halves >> h) & 1)) continue;
               for (int c = 0; c < 2; ++c)
                 tma_load_4d(sm.k[ks] + c * 16384 + h * 8192, &mapK, &sm.k_full[ks], c * 64, sc.g,
-                            kt * 128 + h * 64, sc.b);
+                            sc.k_base + kt * 128 + h * 64, sc.tb);
             }
           }
         } else {
@@ -508,7 +541,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!((need >> h) & 1)) continue;
               for (int c = 0; c < 2; ++c)
                 tma_load_4d(sm.v[vs] + c * 16384 + h * 8192, &mapV, &sm.v_full[vs], c * 64, sc.g,
-                            kt * 128 + h * 64, sc.b);
+                            sc.k_base + kt * 128 + h * 64, sc.tb);
             }
           }
         } else {
@@ -565,6 +598,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int t = 0; t < 2 && ok; ++t) {
             ok = mbar_wait_t(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx, pacc[4]);
             ofph ^= 1u << t;
+            if (ok) mbar_arrive(&sm.o_ack[t]);
           }
           ofree_waited = 3;
           if (!ok) break;
@@ -604,6 +638,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!mbar_wait_t(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx, pacc[4])) return false;
             ofph ^= 1u << t;
             ofree_waited |= 1 << t;
+            mbar_arrive(&sm.o_ack[t]);
             tc_fence_after();
           }
           const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * kKVTileBytes) >> 4);
@@ -679,6 +714,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (!((ofree_waited >> t) & 1)) {
             ok = mbar_wait(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx);
             ofph ^= 1u << t;
+            if (ok) mbar_arrive(&sm.o_ack[t]);
           }
         }
         umma_commit(&sm.q_empty);
@@ -728,9 +764,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int s = 2 * t + ss;
             const int row0 = sc.seg_row0[s];
             // visible query rows row0 + c of this key: c in [lo, hi)
-            int lo = 0, hi = min(64, p.Sq - row0);
-            if (p.causal) lo = max(0, key - row0 - p.causal_off);
-            if (!((mem >> (2 * s + h)) & 1) || key >= p.Sk) hi = 0;
+            int lo = 0, hi = min(64, sc.q_len - row0);
+            if (p.causal) lo = max(0, key - row0 - sc.coff);
+            if (!((mem >> (2 * s + h)) & 1) || key >= sc.k_len) hi = 0;
             float x[64];
             tmem_ld64(lane_base + b * 256 + t * 128 + ss * 64, x);
             float m4[4] = {NEG, NEG, NEG, NEG};
@@ -797,7 +833,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // ---- attention over the unit's blocks (gated: the blocks the gate kept)
       const int my_valid = sc.seg_valid[seg];
       const int my_row = sc.seg_row0[seg] + (r & 63);
-      const bool row_ok = my_valid && my_row < p.Sq;
+      const bool row_ok = my_valid && my_row < sc.q_len;
       float m_used = NEG, l = 0.f;
       int npv = 0;
       auto body = [&](int kt, bool is_col, int mem) -> bool {
@@ -816,14 +852,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int c = 0; c < 64; ++c) {
               const int e = kt * 128 + 64 * h + c;
               bool vis = ((segm >> h) & 1) && e < sc.n_cols && ((sc.colmask[e] >> seg) & 1);
-              if (vis && p.causal) vis = sc.col[e] <= my_row + p.causal_off;
+              if (vis && p.causal) vis = sc.col[e] <= my_row + sc.coff;
               sh[c] = vis ? sh[c] : NEG;
             }
           } else {
             const int key0 = kt * 128 + 64 * h;
             int lim = ((segm >> h) & 1) ? 64 : 0;
-            lim = min(lim, p.Sk - key0);
-            if (p.causal) lim = min(lim, my_row + p.causal_off - key0 + 1);
+            lim = min(lim, sc.k_len - key0);
+            if (p.causal) lim = min(lim, my_row + sc.coff - key0 + 1);
             if (lim < 64) {
 #pragma unroll
               for (int c = 0; c < 64; ++c) sh[c] = (c < lim) ? sh[c] : NEG;
@@ -927,7 +963,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int c = 0; c < 4; ++c) {
           tmem_ld32(lane_addr + 128 + c * 32, ob);
           if (store) {
-            const int64_t off = sc.b * p.osb + static_cast<int64_t>(my_row) * p.oss + head * p.osh + c * 32;
+            const int64_t off = sc.b * p.osb + static_cast<int64_t>(sc.q_base + my_row) * p.oss +
+                                head * p.osh + c * 32;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], inv_l);
             if (p.o_f32) {
@@ -947,7 +984,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       } else if (store) {
-        const int64_t off = sc.b * p.osb + static_cast<int64_t>(my_row) * p.oss + head * p.osh;
+        const int64_t off = sc.b * p.osb + static_cast<int64_t>(sc.q_base + my_row) * p.oss +
+                            head * p.osh;
         for (int c = 0; c < 128; c += 4) {
           if (p.o_f32)
             *reinterpret_cast<float4*>(static_cast<float*>(p.o) + off + c) = make_float4(0, 0, 0, 0);
@@ -956,8 +994,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
       if (store)
-        p.lse[(static_cast<int64_t>(sc.b) * p.Hq + head) * p.Sq + my_row] =
+        p.lse[sc.b * p.lse_sb + head * p.lse_sh + sc.q_base + my_row] =
             l > 0.f ? (m_used + lg2_approx(l)) * 0.69314718055994531f : NEG;
+      // o_free of this unit may complete only after the MMA warp has waited
+      // for the previous unit's (see o_ack)
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_ack[t], n & 1, wctx))) { ok = false; break; }
       tc_fence_before();
       mbar_arrive(&sm.o_free[t]);
       mbar_arrive(&sm.sched_empty[ub]);

@@ -170,8 +170,18 @@ std::atomic<unsigned long long> g_wait_ns{sbfa::kWaitLimitNs};
 // ---------------------------------------------------------------------------
 // prefill launcher (tcgen05 kernel)
 // ---------------------------------------------------------------------------
+// Varlen launches describe the packing here: cu_q / cu_k are the device
+// cumulative lengths (shape B = number of sequences, Sq / Sk = the longest
+// lengths), total_q / total_k the packed row counts of q and k/v.
+struct Varlen {
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
+};
+
 sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sbfa_t4& q,
-                           const sbfa_t4& k, const sbfa_t4& v, cudaStream_t stream) {
+                           const sbfa_t4& k, const sbfa_t4& v, cudaStream_t stream,
+                           const Varlen& vl = Varlen()) {
   DevInfo di;
   SBFA_TRY(dev_info(&di));
   p.B = s->B;
@@ -198,9 +208,21 @@ sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sb
   p.ksb = k.sb; p.kss = k.ss; p.ksh = k.sh;
   p.vsb = v.sb; p.vss = v.ss; p.vsh = v.sh;
   CUtensorMap mq, mk, mv;
-  SBFA_TRY(encode_bshd(&mq, q, s->B, s->Sq, s->Hq, 64));
-  SBFA_TRY(encode_bshd(&mk, k, s->B, s->Sk, s->Hkv, 64));
-  SBFA_TRY(encode_bshd(&mv, v, s->B, s->Sk, s->Hkv, 64));
+  p.cu_q = vl.cu_q;
+  p.cu_k = vl.cu_k;
+  if (vl.cu_q) {
+    SBFA_TRY(encode_bshd(&mq, q, 1, vl.total_q, s->Hq, 64));
+    SBFA_TRY(encode_bshd(&mk, k, 1, vl.total_k, s->Hkv, 64));
+    SBFA_TRY(encode_bshd(&mv, v, 1, vl.total_k, s->Hkv, 64));
+    p.lse_sb = 0;
+    p.lse_sh = vl.total_q;
+  } else {
+    SBFA_TRY(encode_bshd(&mq, q, s->B, s->Sq, s->Hq, 64));
+    SBFA_TRY(encode_bshd(&mk, k, s->B, s->Sk, s->Hkv, 64));
+    SBFA_TRY(encode_bshd(&mv, v, s->B, s->Sk, s->Hkv, 64));
+    p.lse_sb = static_cast<int64_t>(s->Hq) * s->Sq;
+    p.lse_sh = s->Sq;
+  }
   const size_t smem = sizeof(sbfa::PfSmem) + 1024;
   static bool attr_set[64][4] = {};
   int dev = 0;
@@ -684,8 +706,34 @@ sbfa_status sbfa_convert_vertical_slash(const int32_t* q_seqlens, const int32_t*
   const int64_t grid = static_cast<int64_t>(B) * H * nqb;
   sbfa::convert_vs_kernel<<<static_cast<unsigned>(grid), sbfa::kCvThreads, 0,
                             reinterpret_cast<cudaStream_t>(stream)>>>(
-      q_seqlens, kv_seqlens, vertical, nnz_v, slash, nnz_s, H, nqb, block_M, block_N, causal,
-      block_count, block_offset, column_count, column_index, status);
+      q_seqlens, kv_seqlens, vertical, nnz_v, slash, nnz_s, nullptr, nullptr, H, nqb, block_M,
+      block_N, causal, block_count, block_offset, column_count, column_index, status);
+  SBFA_CUDA(cudaGetLastError());
+  return SBFA_OK;
+}
+
+sbfa_status sbfa_convert_vertical_slash_mergehead(
+    const int32_t* q_seqlens, const int32_t* kv_seqlens, const int32_t* vertical, int32_t nnz_v,
+    const int32_t* slash, int32_t nnz_s, const int32_t* vertical_count,
+    const int32_t* slash_count, int32_t B, int32_t H, int32_t context_size, int32_t block_M,
+    int32_t block_N, int32_t causal, int32_t* block_count, int32_t* block_offset,
+    int32_t* column_count, int32_t* column_index, int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  if (!q_seqlens || !kv_seqlens || !vertical || !slash || !vertical_count || !slash_count ||
+      !block_count || !block_offset || !column_count || !column_index)
+    return fail(SBFA_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || H <= 0 || context_size <= 0 || nnz_v < 0 || nnz_s < 0)
+    return fail(SBFA_ERR_INVALID_ARG, "bad sizes");
+  if (block_M != 64 || block_N != 64)
+    return fail(SBFA_ERR_UNSUPPORTED, "block_M = block_N = 64 only");
+  if (context_size > sbfa::kCvMaxWords * 32 * 64)
+    return fail(SBFA_ERR_UNSUPPORTED, "context_size too large");
+  const int nqb = (context_size + block_M - 1) / block_M;
+  const int64_t grid = static_cast<int64_t>(B) * H * nqb;
+  sbfa::convert_vs_kernel<<<static_cast<unsigned>(grid), sbfa::kCvThreads, 0,
+                            reinterpret_cast<cudaStream_t>(stream)>>>(
+      q_seqlens, kv_seqlens, vertical, nnz_v, slash, nnz_s, vertical_count, slash_count, H, nqb,
+      block_M, block_N, causal, block_count, block_offset, column_count, column_index, status);
   SBFA_CUDA(cudaGetLastError());
   return SBFA_OK;
 }
@@ -717,6 +765,77 @@ sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
   p.vs_nqb = (shape->Sq + 63) / 64;
   p.status = status;
   return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Shared checks of the cu_seqlens entry points; fills the shape the
+// launcher sizes its unit grid with (B = sequences, longest lengths).
+static sbfa_status varlen_shape(const int32_t* cu_q, const int32_t* cu_k, int32_t nseq, int32_t total_q,
+                         int32_t total_k, int32_t max_q, int32_t max_k, int32_t Hq, int32_t Hkv,
+                         int32_t D, float scale, int32_t causal, const sbfa_t4& q,
+                         const sbfa_t4& k, const sbfa_t4& v, const sbfa_t4& o, const float* lse,
+                         sbfa_shape* sh) {
+  if (!cu_q || !cu_k) return fail(SBFA_ERR_INVALID_ARG, "cu_seqlens: null pointer");
+  if (nseq <= 0 || total_q <= 0 || total_k <= 0 || max_q <= 0 || max_k <= 0)
+    return fail(SBFA_ERR_INVALID_ARG, "non-positive size");
+  *sh = sbfa_shape{nseq, max_q, max_k, Hq, Hkv, D, scale, causal};
+  SBFA_TRY(check_shape(sh));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  return SBFA_OK;
+}
+
+sbfa_status sbfa_fwd_varlen(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int32_t nseq, int32_t total_q, int32_t total_k,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t Hq, int32_t Hkv,
+                            int32_t D, float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k,
+                            sbfa_t4 v, const sbfa_table* table, sbfa_t4 o, float* lse,
+                            int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  sbfa_shape sh;
+  SBFA_TRY(varlen_shape(cu_seqlens_q, cu_seqlens_k, nseq, total_q, total_k, max_seqlen_q,
+                        max_seqlen_k, Hq, Hkv, D, scale, causal, q, k, v, o, lse, &sh));
+  SBFA_TRY(check_table(table, &sh, true));
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeTable;
+  p.o = o.ptr; p.osb = 0; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.idx = table->idx; p.tsb = table->sb; p.tsh = table->sh; p.tsqb = table->sqb;
+  p.nmax = table->nmax; p.q_block = table->q_block; p.kv_block = table->kv_block;
+  p.status = status;
+  Varlen vl;
+  vl.cu_q = cu_seqlens_q; vl.cu_k = cu_seqlens_k; vl.total_q = total_q; vl.total_k = total_k;
+  return launch_prefill(p, &sh, q, k, v, reinterpret_cast<cudaStream_t>(stream), vl);
+}
+
+sbfa_status sbfa_fwd_vertical_slash_varlen(
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t nseq, int32_t total_q,
+    int32_t total_k, int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t Hq, int32_t Hkv,
+    int32_t D, float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+    const int32_t* block_count, const int32_t* block_offset, int32_t nnz_s,
+    const int32_t* column_count, const int32_t* column_index, int32_t nnz_v, int32_t block_M,
+    int32_t block_N, sbfa_t4 o, float* lse, int32_t* status, sbfa_stream_t stream) {
+  g_last_error.clear();
+  sbfa_shape sh;
+  SBFA_TRY(varlen_shape(cu_seqlens_q, cu_seqlens_k, nseq, total_q, total_k, max_seqlen_q,
+                        max_seqlen_k, Hq, Hkv, D, scale, causal, q, k, v, o, lse, &sh));
+  if (block_M != 64 || block_N != 64)
+    return fail(SBFA_ERR_UNSUPPORTED, "block_M = block_N = 64 only");
+  if (!block_count || !block_offset || !column_count || !column_index)
+    return fail(SBFA_ERR_INVALID_ARG, "null index array");
+  if (nnz_s < 0 || nnz_v < 0) return fail(SBFA_ERR_INVALID_ARG, "negative nnz");
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeVS;
+  p.o = o.ptr; p.osb = 0; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.vs_bc = block_count; p.vs_bo = block_offset; p.nnz_s = nnz_s;
+  p.vs_cc = column_count; p.vs_ci = column_index; p.nnz_v = nnz_v;
+  p.vs_nqb = (max_seqlen_q + 63) / 64;
+  p.status = status;
+  Varlen vl;
+  vl.cu_q = cu_seqlens_q; vl.cu_k = cu_seqlens_k; vl.total_q = total_q; vl.total_k = total_k;
+  return launch_prefill(p, &sh, q, k, v, reinterpret_cast<cudaStream_t>(stream), vl);
 }
 
 size_t sbfa_varlen_selected_workspace_size(int32_t nseq, int32_t total, int32_t max_seqlen,

@@ -242,8 +242,9 @@ sbfa_status sbfa_convert_vertical_slash(const int32_t* q_seqlens, const int32_t*
  * q-block i of head h attends the keys of blocks [off, off + block_N) for
  * the first block_count entries of block_offset, plus the first
  * column_count keys of column_index, with the causal mask if asked.
- * Index arrays as produced by sbfa_convert_vertical_slash (per query head).
- * Requires block_M == block_N == 64, Hq == Hkv.
+ * Index arrays as produced by sbfa_convert_vertical_slash (per query head;
+ * with GQA, query head h reads kv head h / (Hq/Hkv)).  Requires block_M ==
+ * block_N == 64.
  */
 sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
                                     const int32_t* block_count, const int32_t* block_offset,
@@ -251,6 +252,73 @@ sbfa_status sbfa_fwd_vertical_slash(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 
                                     const int32_t* column_index, int32_t nnz_v,
                                     int32_t block_M, int32_t block_N, sbfa_t4 o, float* lse,
                                     int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_convert_vertical_slash_mergehead -- sbfa_convert_vertical_slash with
+ * a per-head number of entries.
+ * Source: Sglang Sparse Flash Attention, Description and Signature
+ * (convert_vertical_slash_indexes_mergehead: per-head variable sparsity
+ * counts vertical_indices_count / slash_indices_count).  Reading taken: the
+ * counts are int32 [H] (device); head h uses the first vertical_count[h] of
+ * its nnz_v vertical entries and the first slash_count[h] of its nnz_s slash
+ * entries (counts are clamped to [0, nnz]); rows are laid out with strides
+ * nnz_v / nnz_s as in sbfa_convert_vertical_slash, whose definition, outputs
+ * and limits apply otherwise.
+ */
+sbfa_status sbfa_convert_vertical_slash_mergehead(
+    const int32_t* q_seqlens, const int32_t* kv_seqlens, const int32_t* vertical, int32_t nnz_v,
+    const int32_t* slash, int32_t nnz_s, const int32_t* vertical_count,
+    const int32_t* slash_count, int32_t B, int32_t H, int32_t context_size, int32_t block_M,
+    int32_t block_N, int32_t causal, int32_t* block_count, int32_t* block_offset,
+    int32_t* column_count, int32_t* column_index, int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_varlen -- block-table attention over sequences packed by
+ * cumulative lengths.
+ * Sources: Flash-Sparse-Attention, Quickstart (cu_seqlens packing of a
+ * variable-length batch); Incremental_FlashAttention README, Usage 1 (the
+ * block table).  Sequence s owns query rows [cu_seqlens_q[s],
+ * cu_seqlens_q[s+1]) of q and key rows [cu_seqlens_k[s], cu_seqlens_k[s+1])
+ * of k and v.  Local query row r of sequence s and head h attends the keys
+ * of the blocks listed in table row idx[s*sb + (h/G)*sh + (r/q_block)*sqb +
+ * n]; entries are block indices local to the sequence (block j = local keys
+ * [j*kv_block, (j+1)*kv_block) clipped to the sequence's key length), with
+ * the sbfa_table rules (padding < 0, repeats count once, entries past the
+ * sequence's last block are skipped and reported).  causal: the bottom-right
+ * mask of each sequence (local key <= r + k_len - q_len).
+ * cu_seqlens_q, cu_seqlens_k: int32 [nseq + 1], device, non-decreasing from
+ * 0; total_q = cu_seqlens_q[nseq], total_k = cu_seqlens_k[nseq] (passed
+ * from the host); max_seqlen_q / max_seqlen_k >= every sequence's length.
+ * q: (1, total_q, Hq, 128) view (sb ignored); k, v: (1, total_k, Hkv, 128);
+ * o like q; lse: fp32 [Hq, total_q].  kv_block in {64, 128, 256}; q_block a
+ * multiple of 64 or >= max_seqlen_q.  No workspace.
+ */
+sbfa_status sbfa_fwd_varlen(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int32_t nseq, int32_t total_q, int32_t total_k,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t Hq, int32_t Hkv,
+                            int32_t D, float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k,
+                            sbfa_t4 v, const sbfa_table* table, sbfa_t4 o, float* lse,
+                            int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_vertical_slash_varlen -- sbfa_fwd_vertical_slash over sequences
+ * packed by cumulative lengths.
+ * Source: Sglang Sparse Flash Attention, Signature and I/O contract
+ * (sparse_attn_varlen_func: cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+ * max_seqlen_k).  The index arrays are those sbfa_convert_vertical_slash
+ * (or its mergehead form) writes with batch = sequence, q_seqlens /
+ * kv_seqlens = the sequence lengths and context_size = max_seqlen_q:
+ * [nseq, Hq, ceil(max_seqlen_q / 64), nnz]; offsets and columns are local to
+ * the sequence.  Packing, layouts, the causal rule and lse as in
+ * sbfa_fwd_varlen; block_M = block_N = 64.
+ */
+sbfa_status sbfa_fwd_vertical_slash_varlen(
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t nseq, int32_t total_q,
+    int32_t total_k, int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t Hq, int32_t Hkv,
+    int32_t D, float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+    const int32_t* block_count, const int32_t* block_offset, int32_t nnz_s,
+    const int32_t* column_count, const int32_t* column_index, int32_t nnz_v, int32_t block_M,
+    int32_t block_N, sbfa_t4 o, float* lse, int32_t* status, sbfa_stream_t stream);
 
 /*
  * sbfa_fwd_varlen_selected -- NSA selected attention over varlen sequences.

@@ -319,7 +319,8 @@ def kept_density_closed_form(n, k_top):
 # ----------------------------------------------------------------------------
 
 def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
-                           block_M, block_N, causal=True, qblocks=None):
+                           block_M, block_N, causal=True, qblocks=None, v_count=None,
+                           s_count=None):
     """Per (b, h, q-block i), rows [m0, m1) with m1 = min(m0 + BM, q_len):
 
     * a slash offset s is the diagonal key = row + (kv_len - q_len) - s; over
@@ -332,7 +333,9 @@ def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
     Entries past the counts are 0.  (Sglang Sparse Flash Attention, I/O
     contract; the aligned-block reading is an assumption.)  ``qblocks``:
     None (every q-block) or the q-block indices to convert; the others are
-    left at count 0."""
+    left at count 0.  ``v_count`` / ``s_count``: None, or per-head numbers
+    of entries in use (convert_vertical_slash_indexes_mergehead: head h reads
+    only the first v_count[h] / s_count[h] entries of its rows)."""
     B, H, nnz_v = vertical.shape
     nnz_s = slash.shape[2]
     nqb = -(-context_size // block_M)
@@ -345,8 +348,10 @@ def convert_vertical_slash(q_seqlens, kv_seqlens, vertical, slash, context_size,
         d = kl - ql
         nkb = -(-kl // block_N)
         for h in range(H):
-            s = slash[b, h].astype(np.int64)
-            vv = vertical[b, h].astype(np.int64)
+            ns = nnz_s if s_count is None else min(max(int(s_count[h]), 0), nnz_s)
+            nv = nnz_v if v_count is None else min(max(int(v_count[h]), 0), nnz_v)
+            s = slash[b, h, :ns].astype(np.int64)
+            vv = vertical[b, h, :nv].astype(np.int64)
             for i in (range(nqb) if qblocks is None else qblocks):
                 m0 = i * block_M
                 if m0 >= ql:
@@ -400,6 +405,50 @@ def attend_vertical_slash(q, k, v, block_count, block_offset, column_count,
                 o[b, r, h, :] = oo
                 lse[b, h, r] = ll
     return o, lse
+
+
+# ----------------------------------------------------------------------------
+# Varlen packing (cu_seqlens): each sequence on its own
+# ----------------------------------------------------------------------------
+
+def _varlen_apply(fn, q, k, v, cu_q, cu_k):
+    """Run fn(q_s, k_s, v_s, s) -> (o (1, Lq, Hq, D), lse (1, Hq, Lq)) on
+    every packed sequence s and pack the results as o (Tq, Hq, D), lse
+    (Hq, Tq) (Flash-Sparse-Attention Quickstart; Sglang sparse_attn_varlen_func:
+    cu_seqlens_q / cu_seqlens_k give each sequence's rows)."""
+    cu_q, cu_k = np.asarray(cu_q, dtype=np.int64), np.asarray(cu_k, dtype=np.int64)
+    Tq, Hq, D = q.shape
+    o = np.full((Tq, Hq, D), np.nan)
+    lse = np.full((Hq, Tq), np.nan)
+    for s in range(len(cu_q) - 1):
+        a, z = cu_q[s], cu_q[s + 1]
+        ka, kz = cu_k[s], cu_k[s + 1]
+        if z == a:
+            continue
+        oo, ll = fn(q[None, a:z], k[None, ka:kz], v[None, ka:kz], s)
+        o[a:z] = oo[0]
+        lse[:, a:z] = ll[0]
+    return o, lse
+
+
+def attend_block_table_varlen(q, k, v, cu_q, cu_k, table, q_block, kv_block, causal, scale):
+    """attend_block_table on each packed sequence: table[s] is its
+    [Hkv, nQB, nmax] table of sequence-local blocks; causal is bottom-right
+    within the sequence."""
+    return _varlen_apply(lambda qs, ks, vs, s: attend_block_table(
+        qs, ks, vs, table[s:s + 1], q_block, kv_block, causal, scale), q, k, v, cu_q, cu_k)
+
+
+def attend_vertical_slash_varlen(q, k, v, cu_q, cu_k, block_count, block_offset, column_count,
+                                 column_index, block_M, block_N, causal, scale):
+    """attend_vertical_slash on each packed sequence with its converted lists
+    (index arrays [nseq, Hq, nQB, nnz], sequence-local offsets and columns)."""
+    def one(qs, ks, vs, s):
+        sl = slice(s, s + 1)
+        return attend_vertical_slash(qs, ks, vs, block_count[sl], block_offset[sl],
+                                     column_count[sl], column_index[sl], block_M, block_N,
+                                     causal, scale)
+    return _varlen_apply(one, q, k, v, cu_q, cu_k)
 
 
 # ----------------------------------------------------------------------------

@@ -617,3 +617,95 @@ def test_nsa_varlen_full_workload_sampled(sb):
     ro, rl = oracle.attend_selected_varlen(wl.q[0], wl.k[0], wl.v[0], cu, sel, 64, True,
                                            wl.scale, rows=lambda h: rows[h])
     compare(o[None], lse[None], ro[None], rl[None], "nsa full")
+
+
+# ------------------------------------------------------------------ varlen (cu_seqlens)
+
+def _cu(lens):
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("causal,q_block,kv_block,G", [(True, 64, 128, 4), (False, 128, 64, 1),
+                                                        (True, 192, 256, 2)])
+def test_fwd_varlen_ragged_sequences(sb, causal, q_block, kv_block, G):
+    """Three packed sequences of different lengths (q_len <= k_len, not
+    multiples of 64), per-sequence tables of sequence-local blocks with
+    padding and a repeat, against the oracle on each sequence alone."""
+    rng = np.random.default_rng(600 + q_block + G)
+    lq, lk = [300, 64, 777], [300, 200, 900]
+    Hkv, nmax = 2, 7
+    Hq = Hkv * G
+    cu_q, cu_k = _cu(lq), _cu(lk)
+    q = W.normal_bf16(rng, (int(cu_q[-1]), Hq, 128))
+    k = W.normal_bf16(rng, (int(cu_k[-1]), Hkv, 128))
+    v = W.normal_bf16(rng, (int(cu_k[-1]), Hkv, 128))
+    nqb = -(-max(lq) // q_block)
+    tab = np.full((3, Hkv, nqb, nmax), -1, np.int32)
+    for s in range(3):
+        nkb = -(-lk[s] // kv_block)
+        for g in range(Hkv):
+            for i in range(-(-lq[s] // q_block)):
+                m = min(nmax - 1, nkb)
+                tab[s, g, i, :m] = rng.choice(nkb, size=m, replace=False)
+    tab[2, 1, 0, -1] = tab[2, 1, 0, 0]        # a repeat counts once
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_varlen(dev(q), dev(k), dev(v), torch.from_numpy(cu_q).cuda(),
+                           torch.from_numpy(cu_k).cuda(), max(lq), max(lk),
+                           torch.from_numpy(tab).cuda(), q_block, kv_block, causal=causal,
+                           status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_block_table_varlen(q, k, v, cu_q, cu_k, tab, q_block, kv_block,
+                                              causal, W.default_scale())
+    compare(o[None], lse[None], ro[None], rl[None], f"varlen table causal={causal} G={G}")
+
+
+def test_vertical_slash_varlen(sb):
+    """sparse_attn_varlen_func: three packed sequences (q_len <= kv_len),
+    lists converted per sequence on the GPU (bit-exact against the oracle),
+    then attention over them."""
+    rng = np.random.default_rng(610)
+    lq, lk = [500, 130, 900], [500, 300, 900]
+    H, nnz_v, nnz_s = 4, 80, 100
+    cu_q, cu_k = _cu(lq), _cu(lk)
+    q = W.normal_bf16(rng, (int(cu_q[-1]), H, 128))
+    k = W.normal_bf16(rng, (int(cu_k[-1]), H, 128))
+    v = W.normal_bf16(rng, (int(cu_k[-1]), H, 128))
+    irng = np.random.default_rng(1610)
+    lists = [W.vertical_slash_indices(irng, 1, H, L, nnz_v, nnz_s) for L in lk]
+    vert = np.concatenate([x[0] for x in lists])
+    slash = np.concatenate([x[1] for x in lists])
+    qs = torch.tensor(lq, dtype=torch.int32, device="cuda")
+    ks = torch.tensor(lk, dtype=torch.int32, device="cuda")
+    g = sb.convert_vertical_slash(qs, ks, torch.from_numpy(vert).cuda(),
+                                  torch.from_numpy(slash).cuda(), max(lq))
+    ref = oracle.convert_vertical_slash(lq, lk, vert, slash, max(lq), 64, 64, True)
+    _check_lists(g, ref)
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_vertical_slash_varlen(dev(q), dev(k), dev(v), torch.from_numpy(cu_q).cuda(),
+                                          torch.from_numpy(cu_k).cuda(), max(lq), max(lk), *g,
+                                          causal=True, status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_vertical_slash_varlen(q, k, v, cu_q, cu_k, *ref, 64, 64, True,
+                                                 W.default_scale())
+    compare(o[None], lse[None], ro[None], rl[None], "vs varlen")
+
+
+def test_convert_vertical_slash_mergehead(sb):
+    """Per-head entry counts (convert_vertical_slash_indexes_mergehead):
+    lists bit-exact against the oracle, then attention over them."""
+    wl = _vs_small(L=2048, H=4, nnz_v=120, nnz_s=160, seed=44)
+    L = wl.q.shape[1]
+    vert, slash = wl.meta["vertical"], wl.meta["slash"]
+    vc = np.array([120, 70, 64, 0], dtype=np.int32)
+    sc = np.array([160, 64, 100, 5], dtype=np.int32)
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    g = sb.convert_vertical_slash_mergehead(sl, sl, torch.from_numpy(vert).cuda(),
+                                            torch.from_numpy(slash).cuda(),
+                                            torch.from_numpy(vc).cuda(),
+                                            torch.from_numpy(sc).cuda(), L)
+    ref = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True, v_count=vc,
+                                        s_count=sc)
+    _check_lists(g, ref)
+    o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), *g, causal=True)
+    ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, *ref, 64, 64, True, wl.scale)
+    compare(o, lse, ro, rl, "vs mergehead")

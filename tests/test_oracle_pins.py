@@ -400,3 +400,73 @@ def test_stored_gated_thresholds_recompute_on_two_heads():
         sm = oracle.block_max_head(wl.q[0, :, h, :], wl.k[0, :, h // 4, :], 64, wl.scale)
         ref = oracle.calibrate_thresholds(sm[None], 64)[0].astype(np.float32)
         np.testing.assert_array_equal(T[h], ref)
+
+
+# ---------------------------------------------------------------- varlen packing and mergehead
+
+def test_varlen_block_table_vs_elementwise_per_sequence():
+    """Packed sequences of different lengths: each sequence's rows equal the
+    element-wise brute force on that sequence alone (bottom-right causal
+    inside the sequence), and rows never see another sequence's keys."""
+    rng = np.random.default_rng(61)
+    D, Hq, Hkv, qbs, kbs, nmax = 8, 4, 2, 16, 8, 5
+    lq, lk = [20, 7, 33], [20, 15, 40]
+    cu_q, cu_k = np.concatenate([[0], np.cumsum(lq)]), np.concatenate([[0], np.cumsum(lk)])
+    q, k, v = _rand(rng, cu_q[-1], Hq, D), _rand(rng, cu_k[-1], Hkv, D), _rand(rng, cu_k[-1], Hkv, D)
+    nqb, nkb = -(-max(lq) // qbs), -(-max(lk) // kbs)
+    table = rng.integers(-1, nkb, size=(3, Hkv, nqb, nmax)).astype(np.int32)
+    for causal in (False, True):
+        o, lse = oracle.attend_block_table_varlen(q, k, v, cu_q, cu_k, table, qbs, kbs, causal, 0.5)
+        for s in range(3):
+            a, z, ka, kz = cu_q[s], cu_q[s + 1], cu_k[s], cu_k[s + 1]
+            mask = oracle.element_mask_from_table(lq[s], lk[s], Hq, Hkv, table[s], qbs, kbs, causal)
+            ob, lb = oracle.attend_dense_masked(q[a:z], k[ka:kz], v[ka:kz], mask, 0.5)
+            np.testing.assert_allclose(o[a:z], ob, rtol=0, atol=1e-12)
+            ls = lse[:, a:z]
+            np.testing.assert_array_equal(np.isneginf(ls), np.isneginf(lb))
+            fin = np.isfinite(lb)
+            np.testing.assert_allclose(ls[fin], lb[fin], rtol=0, atol=1e-12)
+
+
+def test_varlen_vertical_slash_equal_lengths_equal_batched():
+    """Two packed sequences of one length give the batched (B = 2) result."""
+    rng = np.random.default_rng(62)
+    L, H, D, BM = 64, 2, 8, 16
+    q, k, v = _rand(rng, 2, L, H, D), _rand(rng, 2, L, H, D), _rand(rng, 2, L, H, D)
+    vert = np.stack([np.stack([np.sort(rng.choice(L, 6, replace=False)) for _ in range(H)])
+                     for _ in range(2)]).astype(np.int32)
+    slash = np.stack([np.stack([np.sort(rng.choice(L, 5, replace=False)) for _ in range(H)])
+                      for _ in range(2)]).astype(np.int32)
+    lists = oracle.convert_vertical_slash([L, L], [L, L], vert, slash, L, BM, BM, True)
+    ob, lb = oracle.attend_vertical_slash(q, k, v, *lists, BM, BM, True, 0.5)
+    cu = np.array([0, L, 2 * L])
+    ov, lv = oracle.attend_vertical_slash_varlen(q.reshape(2 * L, H, D), k.reshape(2 * L, H, D),
+                                                 v.reshape(2 * L, H, D), cu, cu, *lists, BM, BM,
+                                                 True, 0.5)
+    np.testing.assert_array_equal(ov, ob.reshape(2 * L, H, D))
+    np.testing.assert_array_equal(lv, np.concatenate([lb[0], lb[1]], axis=1))
+
+
+def test_mergehead_counts_truncate_each_head():
+    """Per-head counts: head h's lists equal the element-wise sets of its
+    first v_count[h] vertical and s_count[h] slash entries; full counts give
+    the plain conversion."""
+    rng = np.random.default_rng(63)
+    q_len = kv_len = 120
+    H, nv, ns, BM = 3, 12, 9, 16
+    vert = np.stack([np.sort(rng.choice(kv_len, nv, replace=False)) for _ in range(H)])[None]
+    slash = np.stack([np.sort(rng.choice(kv_len, ns, replace=False)) for _ in range(H)])[None]
+    vert, slash = vert.astype(np.int32), slash.astype(np.int32)
+    vc, sc = np.array([12, 5, 0]), np.array([2, 9, 4])
+    bc, bo, cc, ci = oracle.convert_vertical_slash([q_len], [kv_len], vert, slash, q_len, BM, BM,
+                                                   True, v_count=vc, s_count=sc)
+    for h in range(H):
+        ref = _vs_elementwise(q_len, kv_len, vert[0, h, :vc[h]], slash[0, h, :sc[h]], BM, BM, True)
+        for i, (blocks, cols) in enumerate(ref):
+            assert list(bo[0, h, i, :bc[0, h, i]]) == [b * BM for b in blocks]
+            assert list(ci[0, h, i, :cc[0, h, i]]) == cols
+    full = oracle.convert_vertical_slash([q_len], [kv_len], vert, slash, q_len, BM, BM, True,
+                                         v_count=[nv] * H, s_count=[ns] * H)
+    plain = oracle.convert_vertical_slash([q_len], [kv_len], vert, slash, q_len, BM, BM, True)
+    for a, b in zip(full, plain):
+        np.testing.assert_array_equal(a, b)
