@@ -69,6 +69,9 @@ _SIGS = {
     "sbfa_fwd_vertical_slash_varlen": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                        _I, T4, T4, T4, _P, _P, _I, _P, _P, _I, _I, _I, T4, _P,
                                        _P, _P],
+    "sbfa_fwd_window": [ctypes.POINTER(Shape), T4, T4, T4, _I, T4, _P, _P, _P],
+    "sbfa_fwd_window_varlen": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, T4, T4,
+                               T4, T4, _P, _P, _P],
     "sbfa_fwd_varlen_selected": [_P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, T4, T4, T4, _P,
                                  _I, _I, _P, ctypes.c_size_t, T4, _P, _P, _P],
     "sbfa_varlen_selected_workspace_size": [_I, _I, _I, _I, _I, _I],
@@ -185,6 +188,17 @@ def fwd_dense(q, k, v, causal=False, scale=None, out=None, lse=None, status=None
     shp = _shape(q, k, causal, scale)
     _call("sbfa_fwd_dense", ctypes.byref(shp), _t4(q), _t4(k), _t4(v), _t4(out), lse.data_ptr(),
           _ptr(status), _stream())
+    return out, lse
+
+
+def fwd_window(q, k, v, window, scale=None, out=None, lse=None, status=None):
+    """Causal sliding-window attention of ``window`` keys (``sbfa_fwd_window``).
+    Returns (o, lse)."""
+    _check_bf16(q, k, v)
+    out, lse = _outputs(q, out, lse)
+    shp = _shape(q, k, True, scale)
+    _call("sbfa_fwd_window", ctypes.byref(shp), _t4(q), _t4(k), _t4(v), int(window), _t4(out),
+          lse.data_ptr(), _ptr(status), _stream())
     return out, lse
 
 
@@ -366,6 +380,24 @@ def fwd_vertical_slash_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
           _t4(v[None]), block_count.data_ptr(), block_offset.data_ptr(), block_offset.shape[-1],
           column_count.data_ptr(), column_index.data_ptr(), column_index.shape[-1], block_M,
           block_N, _t4(out[None]), lse.data_ptr(), _ptr(status), _stream())
+    return out, lse
+
+
+def fwd_window_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, window,
+                      scale=None, out=None, lse=None, status=None):
+    """``sbfa_fwd_window_varlen``: causal sliding window over cu_seqlens-packed
+    sequences.  Returns o (total_q, Hq, D), lse (Hq, total_q)."""
+    _check_bf16(q, k, v)
+    nseq, tq, tk = _varlen_args(q, k, cu_seqlens_q, cu_seqlens_k)
+    Hq, D = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, tq, dtype=torch.float32, device=q.device)
+    _call("sbfa_fwd_window_varlen", cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), nseq, tq,
+          tk, int(max_seqlen_q), int(max_seqlen_k), Hq, k.shape[1], D,
+          0.0 if scale is None else float(scale), int(window), _t4(q[None]), _t4(k[None]),
+          _t4(v[None]), _t4(out[None]), lse.data_ptr(), _ptr(status), _stream())
     return out, lse
 
 

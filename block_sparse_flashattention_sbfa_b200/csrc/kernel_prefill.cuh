@@ -84,6 +84,12 @@ struct PrefillParams {
   const int* idx;
   int64_t tsb, tsh, tsqb;
   int nmax, q_block, kv_block, n_kb;
+  // table blocks of 16 or 32 keys: log2(kv_block), else 0; the listed blocks
+  // are then also kept per segment at that granularity (pf_fb) for masking
+  int fine_shift;
+  // dense mode: causal sliding window of this many keys (0: none); row r
+  // sees keys r + causal_off - window < key <= r + causal_off
+  int window;
   // gated mode
   const float* T;
   int nqb;
@@ -109,7 +115,8 @@ struct PrefillParams {
 struct PfSched {
   uint32_t bm[4][kBmWords];  // per segment: 64-key blocks to visit (gated: gate candidates)
   // vertical-slash mode: the unit's column list; gated mode: the same words
-  // hold the keep bitmaps the gate writes ([4][kBmWords], see pf_kb)
+  // hold the keep bitmaps the gate writes ([4][kBmWords], see pf_kb); table
+  // mode with 16- or 32-key blocks: the listed blocks per segment (pf_fb)
   int col[kMaxCols];
   uint8_t colmask[kMaxCols];
   int n_words, n_cols;
@@ -124,6 +131,12 @@ static_assert(kMaxCols >= 4 * kBmWords, "keep bitmaps share the column list's st
 
 __device__ __forceinline__ uint32_t* pf_kb(PfSched& sc) {
   return reinterpret_cast<uint32_t*>(sc.col);
+}
+__device__ __forceinline__ uint32_t* pf_fb(PfSched& sc) {
+  return reinterpret_cast<uint32_t*>(sc.col);
+}
+__device__ __forceinline__ const uint32_t* pf_fb(const PfSched& sc) {
+  return reinterpret_cast<const uint32_t*>(sc.col);
 }
 
 // Pairing slot of the gate's exact block maximum: the two warps that hold
@@ -147,12 +160,10 @@ struct PfSmem {
   uint64_t q_full[2], q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
+  // o_free[t] completes one phase per unit in which tile t ran a PV (its
+  // epilogue has read O), and only then: a tile with no block in a unit
+  // signals nothing, so the phases cannot run ahead of the MMA warp's waits.
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
-  // o_ack[t]: the MMA warp has taken note of tile t's previous o_free phase.
-  // A tile with no block in a unit finishes its epilogue at once; without
-  // this handshake its o_free could complete a second phase before the MMA
-  // warp waits for the first, and the parity test would then wait forever.
-  uint64_t o_ack[2];
   uint64_t ga_full[2], ga_free[2];  // gate: S^T buffers written / read
   uint64_t kb_done;                 // gate: the unit's keep bitmaps are complete
   uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
@@ -224,7 +235,7 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
   const int n_kt = (k_len + 63) / 64;
   const int n_kb = p.mode == kModeTable ? (k_len + p.kv_block - 1) / p.kv_block : 0;
   for (int e = lane; e < 4 * kBmWords; e += 32) (&sc.bm[0][0])[e] = 0u;
-  if (p.mode == kModeGated)
+  if (p.mode == kModeGated || p.fine_shift)
     for (int e = lane; e < 4 * kBmWords; e += 32) pf_kb(sc)[e] = 0u;
   if (lane == 0) {
     sc.n_words = n_words;
@@ -262,9 +273,28 @@ __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int l
     }
     uint32_t* bm = sc.bm[s];
     if (p.mode == kModeDense || p.mode == kModeGated) {
+      // sliding window: the first tile a row of the segment may see
+      int kt_begin = 0;
+      if (p.window > 0) kt_begin = max(0, row0 + coff - p.window + 1) / 64;
       for (int w = lane; w * 32 < kt_end; w += 32) {
-        const int t0 = w * 32, t1 = min(kt_end, t0 + 32);
-        bm[w] = (t1 - t0 == 32) ? 0xffffffffu : ((1u << (t1 - t0)) - 1u);
+        const int t0 = max(w * 32, kt_begin), t1 = min(kt_end, w * 32 + 32);
+        bm[w] = t1 <= t0 ? 0u
+                         : ((t1 - t0 == 32) ? 0xffffffffu : ((1u << (t1 - t0)) - 1u)) << (t0 - w * 32);
+      }
+    } else if (p.mode == kModeTable && p.fine_shift) {
+      // 16- or 32-key blocks: one fine bit per listed block, one coarse bit
+      // per 64-key tile that holds one
+      const int qb = row0 / p.q_block;
+      const int* row = p.idx + b * p.tsb + g * p.tsh + qb * p.tsqb;
+      uint32_t* fb = pf_fb(sc) + s * kBmWords;
+      for (int n = lane; n < p.nmax; n += 32) {
+        const int j = row[n];
+        if (j < 0) continue;
+        if (j >= n_kb) { report(p.status, kDevBadIndex); continue; }
+        const int t = (j << p.fine_shift) >> 6;
+        if (t >= kt_end) continue;
+        atomicOr(&fb[j >> 5], 1u << (j & 31));
+        atomicOr(&bm[t >> 5], 1u << (t & 31));
       }
     } else if (p.mode == kModeTable) {
       const int qb = row0 / p.q_block;
@@ -361,7 +391,11 @@ __device__ __forceinline__ uint32_t pf_q_off(int c, int t) {
   return static_cast<uint32_t>(c * 2 * kQTileBytes / 2 + t * (kQTileBytes / 2));
 }
 
-template <int MODE>
+// EXT: the mask extensions, a sliding window (dense mode) or 16- / 32-key
+// table blocks (table mode); the other instantiations compile without them.
+// VL: sequences packed by cumulative lengths (per-unit bases and lengths are
+// read from the schedule; otherwise they are the launch's constants).
+template <int MODE, bool EXT, bool VL>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
                    const __grid_constant__ CUtensorMap mapK,
@@ -385,7 +419,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.p_full[i], 128);
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.o_free[i], 128);
-      mbar_init(&sm.o_ack[i], 1);
       mbar_init(&sm.ga_full[i], 1);
       mbar_init(&sm.ga_free[i], 8);  // one arrival per softmax warp
     }
@@ -458,7 +491,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!sc.seg_valid[s]) continue;
               for (int c = 0; c < 2; ++c)
                 tma_load_4d(sm.q + pf_q_off(c, t) + h * 8192, &mapQ, &sm.q_full[t], c * 64,
-                            sc.seg_head[s], sc.q_base + sc.seg_row0[s], sc.tb);
+                            sc.seg_head[s], (VL ? sc.q_base : 0) + sc.seg_row0[s], VL ? 0 : sc.b);
             }
           }
         }
@@ -480,7 +513,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!((halves >> h) & 1)) continue;
               for (int c = 0; c < 2; ++c)
                 tma_load_4d(sm.k[ks] + c * 16384 + h * 8192, &mapK, &sm.k_full[ks], c * 64, sc.g,
-                            sc.k_base + kt * 128 + h * 64, sc.tb);
+                            (VL ? sc.k_base : 0) + kt * 128 + h * 64, VL ? 0 : sc.b);
             }
           }
         } else {
@@ -541,7 +574,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!((need >> h) & 1)) continue;
               for (int c = 0; c < 2; ++c)
                 tma_load_4d(sm.v[vs] + c * 16384 + h * 8192, &mapV, &sm.v_full[vs], c * 64, sc.g,
-                            sc.k_base + kt * 128 + h * 64, sc.tb);
+                            (VL ? sc.k_base : 0) + kt * 128 + h * 64, VL ? 0 : sc.b);
             }
           }
         } else {
@@ -575,7 +608,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int ks = 0, vs = 0;
       uint32_t kph = 0, vph = 0;
       uint32_t pph = 0;   // bit t: p_full[t] phase
-      uint32_t ofph = 0;  // bit t: o_free[t] phase
+      uint32_t ofph = 0;  // bit t: parity of the next o_free[t] phase to wait for
+      uint32_t owe = 0;   // bit t: a unit with PV on tile t has not been waited for
+      // before writing tile t's O (or, in the gate, all of TMEM): wait for
+      // the epilogue of the last unit that accumulated into it
+      auto free_o = [&](int t) -> bool {
+        if (!((owe >> t) & 1u)) return true;
+        if (!mbar_wait_t(&sm.o_free[t], (ofph >> t) & 1u, wctx, pacc[4])) return false;
+        ofph ^= 1u << t;
+        owe &= ~(1u << t);
+        return true;
+      };
       int ai = 0;         // gate items issued so far (S^T buffer ai & 1)
       bool ok = true;
       int n = 0;
@@ -591,16 +634,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
              mbar_wait_t(&sm.q_full[1], n & 1, wctx, pacc[5]);
         if (!ok) break;
         int pv_started = 0;    // bit t
-        int ofree_waited = 0;  // bit t
         if (gated) {
           // The gate's S^T buffers cover all of TMEM, O included: the previous
           // unit's epilogue must have read O first.
-          for (int t = 0; t < 2 && ok; ++t) {
-            ok = mbar_wait_t(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx, pacc[4]);
-            ofph ^= 1u << t;
-            if (ok) mbar_arrive(&sm.o_ack[t]);
-          }
-          ofree_waited = 3;
+          ok = free_o(0) && free_o(1);
           if (!ok) break;
           tc_fence_after();
           auto gate = [&](int kt, bool, int) -> bool {
@@ -634,11 +671,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           int valid, act1, f0, v_waited;
         } pend = {0, 0, 0, 0};
         auto issue_pv = [&](int t, int flag) -> bool {
-          if (!((ofree_waited >> t) & 1)) {
-            if (!mbar_wait_t(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx, pacc[4])) return false;
-            ofph ^= 1u << t;
-            ofree_waited |= 1 << t;
-            mbar_arrive(&sm.o_ack[t]);
+          if (!((pv_started >> t) & 1)) {
+            if (!free_o(t)) return false;
             tc_fence_after();
           }
           const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * kKVTileBytes) >> 4);
@@ -710,13 +744,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         ok = pf_for_each<has_cols>(sc, gated ? pf_kb(sc) : &sc.bm[0][0], body);
         if (ok && pend.valid) ok = finish_prev();
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!((ofree_waited >> t) & 1)) {
-            ok = mbar_wait(&sm.o_free[t], ((ofph >> t) & 1u) ^ 1u, wctx);
-            ofph ^= 1u << t;
-            if (ok) mbar_arrive(&sm.o_ack[t]);
-          }
-        }
+        owe |= static_cast<uint32_t>(pv_started);
         umma_commit(&sm.q_empty);
         mbar_arrive(&sm.sched_empty[ub]);
       }
@@ -764,9 +792,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int s = 2 * t + ss;
             const int row0 = sc.seg_row0[s];
             // visible query rows row0 + c of this key: c in [lo, hi)
-            int lo = 0, hi = min(64, sc.q_len - row0);
-            if (p.causal) lo = max(0, key - row0 - sc.coff);
-            if (!((mem >> (2 * s + h)) & 1) || key >= sc.k_len) hi = 0;
+            int lo = 0, hi = min(64, p.Sq - row0);
+            if (p.causal) lo = max(0, key - row0 - p.causal_off);
+            if (!((mem >> (2 * s + h)) & 1) || key >= p.Sk) hi = 0;
             float x[64];
             tmem_ld64(lane_base + b * 256 + t * 128 + ss * 64, x);
             float m4[4] = {NEG, NEG, NEG, NEG};
@@ -833,7 +861,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // ---- attention over the unit's blocks (gated: the blocks the gate kept)
       const int my_valid = sc.seg_valid[seg];
       const int my_row = sc.seg_row0[seg] + (r & 63);
-      const bool row_ok = my_valid && my_row < sc.q_len;
+      const bool row_ok = my_valid && my_row < (VL ? sc.q_len : p.Sq);
+      const int u_coff = VL ? sc.coff : p.causal_off;  // this unit's causal offset
       float m_used = NEG, l = 0.f;
       int npv = 0;
       auto body = [&](int kt, bool is_col, int mem) -> bool {
@@ -852,17 +881,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int c = 0; c < 64; ++c) {
               const int e = kt * 128 + 64 * h + c;
               bool vis = ((segm >> h) & 1) && e < sc.n_cols && ((sc.colmask[e] >> seg) & 1);
-              if (vis && p.causal) vis = sc.col[e] <= my_row + sc.coff;
+              if (vis && p.causal) vis = sc.col[e] <= my_row + u_coff;
               sh[c] = vis ? sh[c] : NEG;
             }
           } else {
             const int key0 = kt * 128 + 64 * h;
             int lim = ((segm >> h) & 1) ? 64 : 0;
-            lim = min(lim, sc.k_len - key0);
-            if (p.causal) lim = min(lim, my_row + sc.coff - key0 + 1);
-            if (lim < 64) {
+            lim = min(lim, (VL ? sc.k_len : p.Sk) - key0);
+            if (p.causal) lim = min(lim, my_row + u_coff - key0 + 1);
+            if (!EXT) {
+              if (lim < 64) {
 #pragma unroll
-              for (int c = 0; c < 64; ++c) sh[c] = (c < lim) ? sh[c] : NEG;
+                for (int c = 0; c < 64; ++c) sh[c] = (c < lim) ? sh[c] : NEG;
+              }
+            } else {
+              // first visible key of a sliding window
+              const int lo = p.window > 0 ? my_row + u_coff - p.window + 1 - key0 : 0;
+              // 16- or 32-key table blocks: which of the half's blocks are listed
+              uint32_t fm = 0xffffffffu;
+              bool part = false;
+              if (p.fine_shift) {
+                const int j0 = key0 >> p.fine_shift;  // first fine block of the half
+                const uint32_t all = (1u << (64 >> p.fine_shift)) - 1u;
+                fm = pf_fb(sc)[seg * kBmWords + (j0 >> 5)] >> (j0 & 31);
+                part = (fm & all) != all;
+              }
+              if (lim < 64 || lo > 0 || part) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                  const bool listed = !p.fine_shift || ((fm >> (c >> p.fine_shift)) & 1u);
+                  sh[c] = (c < lim && c >= lo && listed) ? sh[c] : NEG;
+                }
+              }
             }
           }
         };
@@ -963,8 +1013,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int c = 0; c < 4; ++c) {
           tmem_ld32(lane_addr + 128 + c * 32, ob);
           if (store) {
-            const int64_t off = sc.b * p.osb + static_cast<int64_t>(sc.q_base + my_row) * p.oss +
-                                head * p.osh + c * 32;
+            const int64_t off = sc.b * p.osb + static_cast<int64_t>((VL ? sc.q_base : 0) + my_row) *
+                                p.oss + head * p.osh + c * 32;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], inv_l);
             if (p.o_f32) {
@@ -984,8 +1034,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       } else if (store) {
-        const int64_t off = sc.b * p.osb + static_cast<int64_t>(sc.q_base + my_row) * p.oss +
-                            head * p.osh;
+        const int64_t off = sc.b * p.osb + static_cast<int64_t>((VL ? sc.q_base : 0) + my_row) *
+                            p.oss + head * p.osh;
         for (int c = 0; c < 128; c += 4) {
           if (p.o_f32)
             *reinterpret_cast<float4*>(static_cast<float*>(p.o) + off + c) = make_float4(0, 0, 0, 0);
@@ -994,13 +1044,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
       if (store)
-        p.lse[sc.b * p.lse_sb + head * p.lse_sh + sc.q_base + my_row] =
+        p.lse[sc.b * p.lse_sb + head * p.lse_sh + (VL ? sc.q_base : 0) + my_row] =
             l > 0.f ? (m_used + lg2_approx(l)) * 0.69314718055994531f : NEG;
-      // o_free of this unit may complete only after the MMA warp has waited
-      // for the previous unit's (see o_ack)
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_ack[t], n & 1, wctx))) { ok = false; break; }
-      tc_fence_before();
-      mbar_arrive(&sm.o_free[t]);
+      if (npv > 0) {  // O was read: the MMA warp may write it again
+        tc_fence_before();
+        mbar_arrive(&sm.o_free[t]);
+      }
       mbar_arrive(&sm.sched_empty[ub]);
     }
   }

@@ -224,38 +224,47 @@ sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sb
     p.lse_sh = s->Sq;
   }
   const size_t smem = sizeof(sbfa::PfSmem) + 1024;
-  static bool attr_set[64][4] = {};
+  const bool ext = p.window > 0 || p.fine_shift > 0;
+  if ((p.window > 0 && p.mode != sbfa::kModeDense) || (p.fine_shift && p.mode != sbfa::kModeTable))
+    return fail(SBFA_ERR_INVALID_ARG, "internal: mask extension in the wrong mode");
+  static bool attr_set[64][16] = {};
   int dev = 0;
   SBFA_CUDA(cudaGetDevice(&dev));
+  const bool vl_on = vl.cu_q != nullptr;
   const void* fn = nullptr;
+  // instantiations: table (with or without small blocks, batched or varlen),
+  // dense (plain, window, window varlen), gated, vertical/slash (batched or varlen)
+#define SBFA_PF(M, E, V) reinterpret_cast<const void*>(sbfa::prefill_kernel<M, E, V>)
   switch (p.mode) {
-    case sbfa::kModeTable: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeTable>); break;
-    case sbfa::kModeDense: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeDense>); break;
-    case sbfa::kModeGated: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeGated>); break;
-    case sbfa::kModeVS: fn = reinterpret_cast<const void*>(sbfa::prefill_kernel<sbfa::kModeVS>); break;
+    case sbfa::kModeTable:
+      fn = ext ? (vl_on ? SBFA_PF(sbfa::kModeTable, true, true) : SBFA_PF(sbfa::kModeTable, true, false))
+               : (vl_on ? SBFA_PF(sbfa::kModeTable, false, true) : SBFA_PF(sbfa::kModeTable, false, false));
+      break;
+    case sbfa::kModeDense:
+      if (vl_on && !ext) return fail(SBFA_ERR_INVALID_ARG, "internal: dense varlen without a window");
+      fn = ext ? (vl_on ? SBFA_PF(sbfa::kModeDense, true, true) : SBFA_PF(sbfa::kModeDense, true, false))
+               : SBFA_PF(sbfa::kModeDense, false, false);
+      break;
+    case sbfa::kModeGated:
+      if (vl_on) return fail(SBFA_ERR_INVALID_ARG, "internal: gated varlen");
+      fn = SBFA_PF(sbfa::kModeGated, false, false);
+      break;
+    case sbfa::kModeVS:
+      fn = vl_on ? SBFA_PF(sbfa::kModeVS, false, true) : SBFA_PF(sbfa::kModeVS, false, false);
+      break;
     default: return fail(SBFA_ERR_INVALID_ARG, "internal: bad prefill mode");
   }
-  if (!attr_set[dev][p.mode]) {
+#undef SBFA_PF
+  const int slot = p.mode * 4 + (ext ? 2 : 0) + (vl_on ? 1 : 0);
+  if (!attr_set[dev][slot]) {
     SBFA_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr_set[dev][p.mode] = true;
+    attr_set[dev][slot] = true;
   }
   p.prof = g_prof_counters;
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   const int grid = std::min(p.n_units, di.sms);
-  switch (p.mode) {
-    case sbfa::kModeTable:
-      sbfa::prefill_kernel<sbfa::kModeTable><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
-      break;
-    case sbfa::kModeDense:
-      sbfa::prefill_kernel<sbfa::kModeDense><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
-      break;
-    case sbfa::kModeGated:
-      sbfa::prefill_kernel<sbfa::kModeGated><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
-      break;
-    default:
-      sbfa::prefill_kernel<sbfa::kModeVS><<<grid, sbfa::kPfThreads, smem, stream>>>(mq, mk, mv, p);
-      break;
-  }
+  void* args[] = {&mq, &mk, &mv, &p};
+  SBFA_CUDA(cudaLaunchKernel(fn, dim3(grid), dim3(sbfa::kPfThreads), args, smem, stream));
   SBFA_CUDA(cudaGetLastError());
   return SBFA_OK;
 }
@@ -377,8 +386,12 @@ sbfa_status check_table(const sbfa_table* t, const sbfa_shape* s, bool prefill) 
   if (t->q_block <= 0) return fail(SBFA_ERR_INVALID_ARG, "table: q_block <= 0");
   const int kb = t->kv_block;
   if (prefill) {
-    if (kb != 64 && kb != 128 && kb != 256)
-      return fail(SBFA_ERR_UNSUPPORTED, "kv_block %d (prefill kernel takes 64/128/256)", kb);
+    if (kb != 16 && kb != 32 && kb != 64 && kb != 128 && kb != 256)
+      return fail(SBFA_ERR_UNSUPPORTED, "kv_block %d (16/32/64/128/256)", kb);
+    // 16- and 32-key blocks are tracked one bit each per segment
+    if (kb < 64 && s->Sk > sbfa::kBmWords * 32 * kb)
+      return fail(SBFA_ERR_UNSUPPORTED, "kv_block %d needs Sk <= %d", kb,
+                  sbfa::kBmWords * 32 * kb);
     if (t->q_block % 64 && t->q_block < s->Sq)
       return fail(SBFA_ERR_UNSUPPORTED, "q_block %d: must be a multiple of 64 or >= Sq",
                   t->q_block);
@@ -389,6 +402,18 @@ sbfa_status check_table(const sbfa_table* t, const sbfa_shape* s, bool prefill) 
       return fail(SBFA_ERR_UNSUPPORTED, "nmax %d > %d", t->nmax, sbfa::kDecMaxEntries);
   }
   return SBFA_OK;
+}
+
+// Table fields of the tiled kernel's parameters.
+void set_table(sbfa::PrefillParams& p, const sbfa_table* t, int nmax_override = -1) {
+  p.idx = t->idx;
+  p.tsb = t->sb;
+  p.tsh = t->sh;
+  p.tsqb = t->sqb;
+  p.nmax = nmax_override >= 0 ? nmax_override : t->nmax;
+  p.q_block = t->q_block;
+  p.kv_block = t->kv_block;
+  p.fine_shift = t->kv_block == 16 ? 4 : (t->kv_block == 32 ? 5 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -505,8 +530,7 @@ sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
   p.mode = sbfa::kModeTable;
   p.o = o.ptr; p.osb = o.sb; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
   p.lse = lse;
-  p.idx = table->idx; p.tsb = table->sb; p.tsh = table->sh; p.tsqb = table->sqb;
-  p.nmax = table->nmax; p.q_block = table->q_block; p.kv_block = table->kv_block;
+  set_table(p, table);
   p.n_kb = (shape->Sk + table->kv_block - 1) / table->kv_block;
   p.status = status;
   return launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream));
@@ -556,8 +580,8 @@ sbfa_status sbfa_fwd_partials(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbf
     p.osh = shape->D;
     p.o_f32 = 1;
     p.lse = lse_parts + n * per_l;
-    p.idx = table->idx + n; p.tsb = table->sb; p.tsh = table->sh; p.tsqb = table->sqb;
-    p.nmax = 1; p.q_block = table->q_block; p.kv_block = table->kv_block;
+    set_table(p, table, 1);
+    p.idx = table->idx + n;
     p.n_kb = (shape->Sk + table->kv_block - 1) / table->kv_block;
     p.status = status;
     SBFA_TRY(launch_prefill(p, shape, q, k, v, reinterpret_cast<cudaStream_t>(stream)));
@@ -801,8 +825,50 @@ sbfa_status sbfa_fwd_varlen(const int32_t* cu_seqlens_q, const int32_t* cu_seqle
   p.mode = sbfa::kModeTable;
   p.o = o.ptr; p.osb = 0; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
   p.lse = lse;
-  p.idx = table->idx; p.tsb = table->sb; p.tsh = table->sh; p.tsqb = table->sqb;
-  p.nmax = table->nmax; p.q_block = table->q_block; p.kv_block = table->kv_block;
+  set_table(p, table);
+  p.status = status;
+  Varlen vl;
+  vl.cu_q = cu_seqlens_q; vl.cu_k = cu_seqlens_k; vl.total_q = total_q; vl.total_k = total_k;
+  return launch_prefill(p, &sh, q, k, v, reinterpret_cast<cudaStream_t>(stream), vl);
+}
+
+sbfa_status sbfa_fwd_window(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                            int32_t window, sbfa_t4 o, float* lse, int32_t* status,
+                            sbfa_stream_t stream) {
+  g_last_error.clear();
+  SBFA_TRY(check_shape(shape));
+  SBFA_TRY(check_view(q, "q", true));
+  SBFA_TRY(check_view(k, "k", true));
+  SBFA_TRY(check_view(v, "v", true));
+  SBFA_TRY(check_outputs(o, lse));
+  if (window <= 0) return fail(SBFA_ERR_INVALID_ARG, "window must be positive");
+  sbfa_shape sh = *shape;
+  sh.causal = 1;  // the window is causal
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeDense;
+  p.window = window;
+  p.o = o.ptr; p.osb = o.sb; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
+  p.status = status;
+  return launch_prefill(p, &sh, q, k, v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbfa_status sbfa_fwd_window_varlen(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                   int32_t nseq, int32_t total_q, int32_t total_k,
+                                   int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t Hq,
+                                   int32_t Hkv, int32_t D, float scale, int32_t window, sbfa_t4 q,
+                                   sbfa_t4 k, sbfa_t4 v, sbfa_t4 o, float* lse, int32_t* status,
+                                   sbfa_stream_t stream) {
+  g_last_error.clear();
+  sbfa_shape sh;
+  SBFA_TRY(varlen_shape(cu_seqlens_q, cu_seqlens_k, nseq, total_q, total_k, max_seqlen_q,
+                        max_seqlen_k, Hq, Hkv, D, scale, 1, q, k, v, o, lse, &sh));
+  if (window <= 0) return fail(SBFA_ERR_INVALID_ARG, "window must be positive");
+  sbfa::PrefillParams p{};
+  p.mode = sbfa::kModeDense;
+  p.window = window;
+  p.o = o.ptr; p.osb = 0; p.oss = o.ss; p.osh = o.sh; p.o_f32 = 0;
+  p.lse = lse;
   p.status = status;
   Varlen vl;
   vl.cu_q = cu_seqlens_q; vl.cu_k = cu_seqlens_k; vl.total_q = total_q; vl.total_k = total_k;

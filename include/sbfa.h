@@ -88,10 +88,11 @@ typedef struct {
  * Source: Incremental_FlashAttention README, "What's in this fork" (sparse
  * block-table forward) and Usage 1.  Each query row attends only to the keys
  * of the blocks its table row lists (with the causal mask if shape->causal).
- * Constraints: kv_block in {64, 128, 256}; q_block a multiple of 64 (or
- * >= Sq); Sk <= 524288.  Decode shapes (Sq * Hq/Hkv <= 16 and one q-block)
- * that are not causal, or have Sq = 1, run on the split-KV decode kernel,
- * which also takes kv_block 16 and 32.
+ * Constraints: kv_block in {16, 32, 64, 128, 256} (README, "What's in this
+ * fork": block sizes at hdim 128); Sk <= 524288, and Sk <= 8192 * kv_block
+ * for 16- and 32-key blocks; q_block a multiple of 64 (or >= Sq).  Decode
+ * shapes (Sq * Hq/Hkv <= 16 and one q-block) that are not causal, or have
+ * Sq = 1, run on the split-KV decode kernel; the rest on the tiled kernel.
  * Outputs: o (bf16, like q), lse (fp32 [B, Hq, Sq]).
  * status: optional device int32, SBFA_DEV_* bits are ORed in.
  */
@@ -106,6 +107,19 @@ sbfa_status sbfa_fwd(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
  */
 sbfa_status sbfa_fwd_dense(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
                            sbfa_t4 o, float* lse, int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_window -- causal sliding-window attention.
+ * Source: Flash-Sparse-Attention, Quickstart (window_size = 512: NSA's
+ * sliding-window branch, here on its own, returning (o, lse)).  Row r
+ * attends the keys r + (Sk - Sq) - window < key <= r + (Sk - Sq)
+ * (bottom-right causal; shape->causal is ignored).  window >= 1.  Same
+ * layouts and limits as sbfa_fwd_dense; runs on the tiled kernel, whose
+ * schedule visits only the key tiles inside each q-block's window.
+ */
+sbfa_status sbfa_fwd_window(const sbfa_shape* shape, sbfa_t4 q, sbfa_t4 k, sbfa_t4 v,
+                            int32_t window, sbfa_t4 o, float* lse, int32_t* status,
+                            sbfa_stream_t stream);
 
 /*
  * sbfa_fwd_partials -- one (o, lse) per table entry.
@@ -299,6 +313,18 @@ sbfa_status sbfa_fwd_varlen(const int32_t* cu_seqlens_q, const int32_t* cu_seqle
                             int32_t D, float scale, int32_t causal, sbfa_t4 q, sbfa_t4 k,
                             sbfa_t4 v, const sbfa_table* table, sbfa_t4 o, float* lse,
                             int32_t* status, sbfa_stream_t stream);
+
+/*
+ * sbfa_fwd_window_varlen -- sbfa_fwd_window over sequences packed by
+ * cumulative lengths (the window and the causal offset are per sequence).
+ * Packing, layouts and lse as in sbfa_fwd_varlen.
+ */
+sbfa_status sbfa_fwd_window_varlen(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                   int32_t nseq, int32_t total_q, int32_t total_k,
+                                   int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t Hq,
+                                   int32_t Hkv, int32_t D, float scale, int32_t window, sbfa_t4 q,
+                                   sbfa_t4 k, sbfa_t4 v, sbfa_t4 o, float* lse, int32_t* status,
+                                   sbfa_stream_t stream);
 
 /*
  * sbfa_fwd_vertical_slash_varlen -- sbfa_fwd_vertical_slash over sequences

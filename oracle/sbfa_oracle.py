@@ -408,6 +408,39 @@ def attend_vertical_slash(q, k, v, block_count, block_offset, column_count,
 
 
 # ----------------------------------------------------------------------------
+# Causal sliding window (NSA's window branch, Flash-Sparse-Attention Quickstart)
+# ----------------------------------------------------------------------------
+
+def attend_window(q, k, v, window, scale, rows=None):
+    """Row r attends the keys r + (Sk - Sq) - window < key <= r + (Sk - Sq)
+    (bottom-right causal window of ``window`` keys ending at the row's own
+    position).  Shapes and ``rows`` as in attend_block_table."""
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    off = Sk - Sq
+    o = np.full((B, Sq, Hq, D), np.nan)
+    lse = np.full((B, Hq, Sq), np.nan)
+    for b in range(B):
+        for h in range(Hq):
+            rr = np.arange(Sq) if rows is None else np.asarray(rows(b, h))
+            for r in rr:
+                hi = r + off                       # last visible key
+                keys = np.arange(max(0, hi - window + 1), min(Sk, hi + 1))
+                oo, ll = attend_keyset(q[b, r:r + 1, h, :], k[b, keys, h // G, :],
+                                       v[b, keys, h // G, :], None, scale)
+                o[b, r, h, :] = oo[0]
+                lse[b, h, r] = ll[0]
+    return o, lse
+
+
+def attend_window_varlen(q, k, v, cu_q, cu_k, window, scale):
+    """attend_window on each packed sequence."""
+    return _varlen_apply(lambda qs, ks, vs, s: attend_window(qs, ks, vs, window, scale),
+                         q, k, v, cu_q, cu_k)
+
+
+# ----------------------------------------------------------------------------
 # Varlen packing (cu_seqlens): each sequence on its own
 # ----------------------------------------------------------------------------
 

@@ -709,3 +709,58 @@ def test_convert_vertical_slash_mergehead(sb):
     o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(wl.k), dev(wl.v), *g, causal=True)
     ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, *ref, 64, 64, True, wl.scale)
     compare(o, lse, ro, rl, "vs mergehead")
+
+
+# ------------------------------------------------------------------ sliding window, small blocks
+
+@pytest.mark.parametrize("Sq,Sk,window,G", [(2048, 2048, 512, 4), (700, 1000, 100, 1)])
+def test_sliding_window(sb, Sq, Sk, window, G):
+    """NSA's window branch (window 512 in the FSA Quickstart), and a window
+    that is not a multiple of 64 with q_len < kv_len; all rows checked."""
+    rng = np.random.default_rng(620 + window)
+    Hkv = 2
+    q = W.normal_bf16(rng, (1, Sq, Hkv * G, 128))
+    k = W.normal_bf16(rng, (1, Sk, Hkv, 128))
+    v = W.normal_bf16(rng, (1, Sk, Hkv, 128))
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_window(dev(q), dev(k), dev(v), window, status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_window(q, k, v, window, W.default_scale())
+    compare(o, lse, ro, rl, f"window {window} Sq={Sq} Sk={Sk}")
+
+
+def test_sliding_window_varlen(sb):
+    rng = np.random.default_rng(630)
+    lq, lk = [900, 64, 1300], [900, 300, 1300]
+    Hq, Hkv = 4, 2
+    cu_q, cu_k = _cu(lq), _cu(lk)
+    q = W.normal_bf16(rng, (int(cu_q[-1]), Hq, 128))
+    k = W.normal_bf16(rng, (int(cu_k[-1]), Hkv, 128))
+    v = W.normal_bf16(rng, (int(cu_k[-1]), Hkv, 128))
+    o, lse = sb.fwd_window_varlen(dev(q), dev(k), dev(v), torch.from_numpy(cu_q).cuda(),
+                                  torch.from_numpy(cu_k).cuda(), max(lq), max(lk), 512)
+    ro, rl = oracle.attend_window_varlen(q, k, v, cu_q, cu_k, 512, W.default_scale())
+    compare(o[None], lse[None], ro[None], rl[None], "window varlen")
+
+
+@pytest.mark.parametrize("kv_block,causal", [(16, True), (32, False), (16, False), (32, True)])
+def test_block_table_small_blocks_tiled(sb, kv_block, causal):
+    """Table blocks of 16 and 32 keys (README: block_size in {16, 32, 64,
+    128, 256} at hdim 128) on the tiled kernel, Sq = Sk = 2048, GQA 4, with
+    padding and a repeat."""
+    rng = np.random.default_rng(640 + kv_block + causal)
+    S, Hkv, G, nmax = 2048, 2, 4, 40
+    q = W.normal_bf16(rng, (1, S, Hkv * G, 128))
+    k = W.normal_bf16(rng, (1, S, Hkv, 128))
+    v = W.normal_bf16(rng, (1, S, Hkv, 128))
+    nkb = S // kv_block
+    tab = np.stack([np.stack([rng.choice(nkb, size=nmax, replace=False) for _ in range(S // 64)])
+                    for _ in range(Hkv)])[None].astype(np.int32)
+    tab[..., -3:] = -1
+    tab[..., -4] = tab[..., 0]
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd(dev(q), dev(k), dev(v), torch.from_numpy(tab).cuda(), 64, kv_block,
+                    causal=causal, status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_block_table(q, k, v, tab, 64, kv_block, causal, W.default_scale())
+    compare(o, lse, ro, rl, f"kv_block {kv_block} causal={causal}")

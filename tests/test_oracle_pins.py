@@ -470,3 +470,25 @@ def test_mergehead_counts_truncate_each_head():
     plain = oracle.convert_vertical_slash([q_len], [kv_len], vert, slash, q_len, BM, BM, True)
     for a, b in zip(full, plain):
         np.testing.assert_array_equal(a, b)
+
+
+def test_window_vs_elementwise_and_full_window_equals_causal():
+    rng = np.random.default_rng(64)
+    B, Sq, Sk, Hq, Hkv, D = 1, 30, 45, 4, 2, 8
+    q, k, v = _rand(rng, B, Sq, Hq, D), _rand(rng, B, Sk, Hkv, D), _rand(rng, B, Sk, Hkv, D)
+    w = 7
+    o, lse = oracle.attend_window(q, k, v, w, 0.5)
+    mask = np.zeros((Hq, Sq, Sk), dtype=bool)
+    for h in range(Hq):
+        for r in range(Sq):
+            for c in range(Sk):
+                mask[h, r, c] = (r + (Sk - Sq) - w) < c <= r + (Sk - Sq)
+    ob, lb = oracle.attend_dense_masked(q[0], k[0], v[0], mask, 0.5)
+    np.testing.assert_allclose(o[0], ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[0], lb, rtol=0, atol=1e-12)
+    # a window as long as the keys is plain causal attention
+    ow, lw = oracle.attend_window(q, k, v, Sk, 0.5)
+    full = np.broadcast_to(np.arange(Sk // 5, dtype=np.int32), (B, Hkv, 1, Sk // 5))
+    oc, lc = oracle.attend_block_table(q, k, v, full, Sq, 5, True, 0.5)
+    np.testing.assert_allclose(ow, oc, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lw, lc, rtol=0, atol=1e-12)
