@@ -4,7 +4,10 @@
 //
 // Work layout: every (batch b, kv-head g) pair owns a fixed run of `pp`
 // chunk slots of 64 keys -- the dense source A (k_spec/v_spec) cut into
-// chunks, then kv_block/64 slots per table entry of source B (k/v).  The
+// chunks and kv_block/64 slots per table entry of source B (k/v), the A
+// chunks spread evenly among the B ones (dec_slot): the dense range is the
+// same keys of every pair and streams more slowly than the scattered table
+// blocks, so a CTA whose range held mostly A chunks used to finish last.  The
 // slots of all pairs are laid end to end and CTA c of the persistent grid
 // takes the contiguous range [total*c/grid, total*(c+1)/grid): the split is
 // known at launch, so no CTA scans the table before streaming.  A table
@@ -41,6 +44,7 @@ constexpr int kDecMaxEntries = 1024;
 constexpr int kDecRows = 16;
 constexpr int kDecD = 128;
 constexpr int kDecSharers = 8;  // sharers of a pair listed ahead of time
+constexpr int kDecStashRows = 7;  // rows a warp can park in the merge buffer (see stash)
 
 struct DecodeParams {
   int B, Sq, Hq, Hkv, G, rows;
@@ -75,6 +79,8 @@ struct DecSmem {
   float lw[kDecGroupWarps][kDecRows];
   int2 meta[kDecWarps][kDecWarpStages];  // slice in each stage: {key0, nk | src << 7 | pr << 8}
   uint32_t repeat[kDecWarps][2];         // repeat masks of a warp's even / odd chunk windows
+  float stm[kDecWarps][kDecStashRows];   // parked first-piece state: running max, sum
+  float stl[kDecWarps][kDecStashRows];
   int last[2];                           // this CTA finishes shared pair 0 / 1
   // CTAs sharing this CTA's first / last pair: their partial slots (-1 for
   // an empty range) when there are at most kDecSharers of them, and count
@@ -84,9 +90,21 @@ struct DecSmem {
 };
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decode shared memory exceeds 227 KB");
+static_assert(kDecWarps * kDecStashRows * kDecD <= kDecGroupWarps * kDecRows * kDecD,
+              "parked first-piece states must fit the merge buffer");
 
 __device__ __forceinline__ int dec_chunks_per_entry(int kv_block) {
   return kv_block >= kDecChunk ? kv_block / kDecChunk : 1;
+}
+
+// Slot c of a pair's pp slots: an A chunk (isA, its index a) or a B chunk
+// (its index c - a among the B slots).  A chunk a sits at the slot where
+// floor(c * nA / pp) steps up.
+__device__ __forceinline__ bool dec_slot(int c, int nA, int pp, int& idx) {
+  const int a = static_cast<int>((static_cast<int64_t>(c) * nA) / pp);
+  const bool isA = static_cast<int>((static_cast<int64_t>(c + 1) * nA) / pp) > a;
+  idx = isA ? a : c - a;
+  return isA;
 }
 
 __device__ __forceinline__ int64_t dec_range_lo(int c, int64_t total, int grid) {
@@ -176,10 +194,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     N = hi - lo;
   }
   if (N == 0) return;
+  const int pr_first = static_cast<int>(lo / pp), pr_last = static_cast<int>((hi - 1) / pp);
+  // A range that ends one pair and starts the next runs its longer piece
+  // first: merging a short leading piece stops all warps early in the stream,
+  // while DRAM is busiest, and that stall used to make such CTAs finish last.
+  // Sequence position 0 is then slot lo + rot and the range wraps around.
+  int64_t rot = 0;
+  if (!p.pair_mode && n_pieces == 2) {
+    const int64_t first_len = static_cast<int64_t>(pr_first + 1) * pp - lo;
+    if (first_len < N - first_len) rot = first_len;
+  }
   // global slot of sequence position n
   auto seq_x = [&](int64_t n) -> int64_t {
     if (p.pair_mode) return (cta + (n / pp) * grid) * static_cast<int64_t>(pp) + n % pp;
-    return lo + n;
+    const int64_t m = n + rot;
+    return lo + (m < N ? m : m - N);
   };
 
   const int grp = warp / kDecGroupWarps, wg = warp % kDecGroupWarps;
@@ -195,13 +224,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     if (j < n_mine) {
       const int64_t x = seq_x(grp + 2 * static_cast<int64_t>(j));
       const int pr = static_cast<int>(x / pp), c = static_cast<int>(x % pp);
-      int nk = 0, src = 0;
-      if (c < nA) {
-        key0 = c * kDecChunk;
+      int nk = 0, src = 0, si;
+      if (dec_slot(c, nA, pp, si)) {
+        key0 = si * kDecChunk;
         nk = min(kDecChunk, p.S_A - key0);
       } else {
         src = 1;
-        const int e = (c - nA) / cpe, sub = (c - nA) % cpe;
+        const int e = si / cpe, sub = si % cpe;
         const int b = pr / p.Hkv, g = pr % p.Hkv;
         const int jb = __ldg(p.idx + b * p.tsb + g * p.tsh + e);
         if (jb >= 0 && jb < p.n_kb) {
@@ -231,9 +260,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     if (j < n_mine) {
       const int64_t x = seq_x(grp + 2 * static_cast<int64_t>(j));
       const int c = static_cast<int>(x % pp);
-      if (c >= nA) {
+      int si;
+      if (!dec_slot(c, nA, pp, si)) {
         pr = static_cast<int>(x / pp);
-        e = (c - nA) / cpe;
+        e = si / cpe;
         jb = __ldg(p.idx + (pr / p.Hkv) * p.tsb + (pr % p.Hkv) * p.tsh + e);
         if (jb >= p.n_kb) jb = -1;
       }
@@ -307,7 +337,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
 
   // pair of piece pi
   auto piece_pair = [&](int pi) {
-    return p.pair_mode ? cta + pi * grid : static_cast<int>(lo / pp) + pi;
+    if (p.pair_mode) return cta + pi * grid;
+    if (rot) return pi == 0 ? pr_last : pr_first;
+    return static_cast<int>(lo / pp) + pi;
   };
   // Rows r0 = gq and r1 = gq + 8 of the M = 16 tile (row = sq * G + head in group)
   // and their causal limits in source A (bottom-right aligned).
@@ -334,16 +366,44 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     }
   };
 
-  load_q(piece_pair(0));
+  // Pull the query rows of pair pr into L2 ahead of their load_q: at a piece
+  // boundary the next piece's Q would otherwise cost a DRAM round trip with
+  // the whole CTA waiting.  Lane l takes 128-byte line l of the <= 16 rows.
+  auto prefetch_q = [&](int pr) {
+    const int rr = lane >> 1;
+    if (rr < p.rows) {
+      const int b = pr / p.Hkv, g = pr % p.Hkv;
+      const __nv_bfloat16* a =
+          p.q + b * p.qsb + (rr / p.G) * p.qss + (g * p.G + rr % p.G) * p.qsh + (lane & 1) * 64;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+    }
+  };
+
+  // the table read and the first copies go out before the Q loads: the
+  // copies need the table, Q is needed only once they land
   load_meta(0);
 #pragma unroll
   for (int s = 0; s < kDecWarpStages; ++s) issue(s);
+  load_q(piece_pair(0));
+  // the query rows of the CTA's next pieces travel with the first copies
+  if (warp >= 1 && warp < 4 && warp < n_pieces) prefetch_q(piece_pair(warp));
+  // Touch the partial slots of this CTA's shared pairs early: the CTA that
+  // merges a pair at the end reads the other sharers' slots, and a cold
+  // address translation there cost several microseconds at the very end.
+  if (!p.pair_mode && warp == 4 && lane < 2 * kDecSharers) {
+    const int k = lane / kDecSharers;
+    const int pr = k == 0 ? pr_first : pr_last;
+    const int cc = dec_cta_of(static_cast<int64_t>(pr) * pp, total, grid) + lane % kDecSharers;
+    if (cc < grid) {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ws_part + static_cast<int64_t>(2 * cc) * kDecRows * kDecD));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ws_lse + 2 * cc * kDecRows));
+    }
+  }
   if (DEDUP) load_dup(0);
 
   // While the first copies are in flight: which CTAs share this CTA's first
   // and last pair, and the partial slot each of them writes (the 64-bit
   // divisions stay off the end of the kernel).
-  const int pr_first = static_cast<int>(lo / pp), pr_last = static_cast<int>((hi - 1) / pp);
   if (!p.pair_mode && warp == kDecWarps - 1 && lane < 2 * kDecSharers) {
     const int k = lane / kDecSharers, s = lane % kDecSharers;
     const int pr = k == 0 ? pr_first : pr_last;
@@ -363,6 +423,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     }
   }
 
+  // A two-piece range with at most kDecStashRows query rows does not stop
+  // its warps between the pieces: each warp parks its state for the first
+  // piece in the merge buffer (no barrier) and streams on; the parked states
+  // are merged once at the end, before the last piece's merge reuses the
+  // buffer.  Larger row counts merge between the pieces.
+  const bool stash = !p.pair_mode && n_pieces == 2 && p.rows <= kDecStashRows;
+  float* const sto = &sm.ow[0][0][0];  // parked O: [warp][row < kDecStashRows][d]
+
   // running state of the piece in progress
   float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
   float oacc[16][4];
@@ -379,11 +447,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       whole = true;
     } else {
       const int64_t a = static_cast<int64_t>(pr) * pp, e = a + pp;
-      nb = (a > lo ? a : lo) - lo;
-      ne = (e < hi ? e : hi) - lo;
+      const int64_t sb = a > lo ? a : lo, se = e < hi ? e : hi;  // its slots
+      nb = sb - lo - rot;
+      if (nb < 0) nb += N;
+      ne = nb + (se - sb);
       whole = a >= lo && e <= hi;
     }
     const int b = pr / p.Hkv, g = pr % p.Hkv;
+    if (pi + 4 < n_pieces && warp == 0) prefetch_q(piece_pair(pi + 4));
     m0 = m1 = NEG;
     l0 = l1 = 0.f;
 #pragma unroll
@@ -490,6 +561,52 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (stash && pi == 0) {
+      // park the first piece (rows < kDecStashRows: only row r0 = gq is live)
+      if (v0) {
+        if (cq == 0) {
+          sm.stm[warp][gq] = m0;
+          sm.stl[warp][gq] = l0;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          *reinterpret_cast<float2*>(sto + (warp * kDecStashRows + gq) * kDecD + i * 8 + 2 * cq) =
+              make_float2(oacc[i][0], oacc[i][1]);
+      }
+      continue;
+    }
+    if (stash) {
+      // every warp has parked the first piece: merge its eight states
+      __syncthreads();
+      const int pr0 = piece_pair(0);
+      const int b0 = pr0 / p.Hkv, g0 = pr0 % p.Hkv;
+      const int64_t a0 = static_cast<int64_t>(pr0) * pp;
+      const bool whole0 = a0 >= lo && a0 + pp <= hi;
+      const int slot0 = (pr0 == pr_first) ? 2 * cta : 2 * cta + 1;
+      const int d = tid % kDecD;
+      for (int rr = tid / kDecD; rr < p.rows; rr += 2) {
+        float M = NEG;
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm.stm[w][rr]);
+        const float Mu = (M == NEG) ? 0.f : M;
+        float L = 0.f, acc = 0.f;
+        for (int w = 0; w < kDecWarps; ++w) {
+          const float wt = ex2_approx(sm.stm[w][rr] - Mu);
+          L += wt * sm.stl[w][rr];
+          acc += wt * sto[(w * kDecStashRows + rr) * kDecD + d];
+        }
+        const float ov = L > 0.f ? acc / L : 0.f;
+        const float lv = L > 0.f ? (Mu + lg2_approx(L)) * 0.69314718055994531f : NEG;
+        const int sq = rr / p.G, h = g0 * p.G + rr % p.G;
+        if (whole0) {
+          p.o[b0 * p.osb + sq * p.oss + h * p.osh + d] = __float2bfloat16(ov);
+          if (d == 0) p.lse[(static_cast<int64_t>(b0) * p.Hq + h) * p.Sq + sq] = lv;
+        } else {
+          p.ws_part[(static_cast<int64_t>(slot0) * kDecRows + rr) * kDecD + d] = ov;
+          if (d == 0) p.ws_lse[slot0 * kDecRows + rr] = lv;
+        }
+      }
+      __syncthreads();  // the parked states are read: the buffer is free below
+    }
     // (1) group 1 publishes its state, group 0 folds it into its registers
     if (grp == 1) {
       if (cq == 0) {
@@ -544,7 +661,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       // 256 threads: thread t owns column d = t % 128 of rows r with r % 2 == t / 128
       const int d = tid % kDecD;
       const int rpar = tid / kDecD;
-      const int slot = (pi == 0) ? 2 * cta : 2 * cta + 1;
+      const int slot = (pr == pr_first) ? 2 * cta : 2 * cta + 1;
       for (int rr = rpar; rr < p.rows; rr += 2) {
         float M = NEG;
         for (int w = 0; w < kDecGroupWarps; ++w) M = fmaxf(M, sm.mw[w][rr]);
@@ -586,17 +703,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     return n;
   };
   if (tid == 0) {
-    // One ticket per shared pair.  The add releases this CTA's partials (the
-    // barrier before it orders every thread's writes ahead of it) and, for
-    // the last taker, acquires those of the other sharers.
-    const int ticket0 = split0 ? atom_add_acq_rel_gpu(p.ws_ticket + pr_first, 1) : 0;
-    const int ticket1 = split1 ? atom_add_acq_rel_gpu(p.ws_ticket + pr_last, 1) : 0;
+    // One ticket per shared pair.  The fence releases this CTA's partials
+    // (the barrier before it orders every thread's writes ahead of it); the
+    // two adds are relaxed, so they travel together; the last taker's
+    // second fence acquires the other sharers' partials.
+    fence_acq_rel_gpu();
+    const int ticket0 = split0 ? atom_add_relaxed_gpu(p.ws_ticket + pr_first, 1) : 0;
+    const int ticket1 = split1 ? atom_add_relaxed_gpu(p.ws_ticket + pr_last, 1) : 0;
     sm.last[0] = split0 && ticket0 == ctas_sharing(0, pr_first) - 1;
     sm.last[1] = split1 && ticket1 == ctas_sharing(1, pr_last) - 1;
+    if (sm.last[0] || sm.last[1]) fence_acq_rel_gpu();
   }
   __syncthreads();
+  // when this CTA finishes both of its shared pairs, warps 0-3 merge the
+  // first and warps 4-7 the second, side by side
+  const bool both = sm.last[0] && sm.last[1];
   for (int k = 0; k < 2; ++k) {
     if (!sm.last[k]) continue;
+    if (both && (warp >> 2) != k) continue;
     const int pr = k == 0 ? pr_first : pr_last;
     const int b = pr / p.Hkv, g = pr % p.Hkv;
     const bool many = sm.share_many[k];
@@ -607,7 +731,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
     }
     const int d4 = (tid & 31) * 4;
     // one warp per row, four columns per lane; partials fetched four CTAs at a time
-    for (int rr = warp; rr < p.rows; rr += kDecWarps) {
+    const int w0 = both ? (warp & 3) : warp, ws = both ? 4 : kDecWarps;
+    for (int rr = w0; rr < p.rows; rr += ws) {
       float M = NEG, W = 0.f;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       for (int c0 = c_first; c0 <= c_last; c0 += 4) {
@@ -660,7 +785,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodePara
       if (lane == 0)
         p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.Sq + sq] = W > 0.f ? M + __logf(W) : NEG;
     }
-    if (tid == 0) p.ws_ticket[pr] = 0;
+    if (tid == (both ? 128 * k : 0)) p.ws_ticket[pr] = 0;
   }
 }
 

@@ -32,12 +32,17 @@ __device__ __forceinline__ void report(int* status, int bit) {
   if (status) atomicOr(status, bit);
 }
 
-// Fetch-and-add at GPU scope with acquire-release semantics: releases this
-// thread's prior writes (and, after a CTA barrier, those of its CTA) and
-// acquires the writes released by earlier adds on the same word.
-__device__ __forceinline__ int atom_add_acq_rel_gpu(int* ptr, int v) {
+// Fence at GPU scope with acquire-release semantics: after a CTA barrier it
+// releases the CTA's prior writes to later operations of this thread, and
+// acquires what other threads released before the atomics it follows.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Relaxed fetch-and-add at GPU scope (ordering comes from the fences).
+__device__ __forceinline__ int atom_add_relaxed_gpu(int* ptr, int v) {
   int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
   return old;
 }
 
