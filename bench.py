@@ -335,7 +335,7 @@ def vs_flops(bc, bo, cc, ci, L, block=64):
 
 
 def bench_vs(torch, sb, dist, args, flush, peaks, peak_kind):
-    wl = W.make_vertical_slash()
+    wl = W.make_vertical_slash(L=args.vs_len)
     L = wl.q.shape[1]
     q, k, v = (W.to_torch_bf16(x, "cuda") for x in (wl.q, wl.k, wl.v))
     sl = torch.tensor([L], dtype=torch.int32, device="cuda")
@@ -353,7 +353,7 @@ def bench_vs(torch, sb, dist, args, flush, peaks, peak_kind):
     cms, _ = time_device(torch, dist, conv, steps, 1, flush)
     tf = flops / (ms * 1e-3) / 1e12
     dense = 4 * 128 * 32 * L * (L + 1) // 2
-    res = {"workload": "vertical-slash prefill B=1 H=32 L=131072 causal D=128 bf16 "
+    res = {"workload": f"vertical-slash prefill B=1 H=32 L={L} causal D=128 bf16 "
                        "BM=BN=64, 1000 vertical + 6000 slash per head",
            "ms": round(ms, 3), "tflops": round(tf, 2), "flops": flops,
            "frac_of_causal_dense": round(flops / dense, 4),
@@ -588,6 +588,8 @@ def main():
                     help="comma-separated prefill workloads to time after the headline, or none")
     ap.add_argument("--gated-len", type=int, default=32768,
                     help="sequence length of the gated workload (a multiple of 64, <= 32768)")
+    ap.add_argument("--vs-len", type=int, default=131072,
+                    help="sequence length of the vertical-slash workload (profiling runs use less)")
     ap.add_argument("--nsa-seqlens", default="65536,32768",
                     help="sequence lengths of the NSA varlen workload")
     ap.add_argument("--no-cpu-baseline", action="store_true",

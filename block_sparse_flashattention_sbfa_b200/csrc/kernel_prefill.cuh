@@ -69,6 +69,12 @@ struct PrefillParams {
   int B, Sq, Sk, Hq, Hkv, G;
   int hp, subs_per_unit, n_sub, n_hgrp, n_subgrp, n_units, n_kt;
   int causal, causal_off;
+  // unit order: 0 = by q-block group, heaviest first, across heads; 1 = head
+  // by head, heaviest group first within a head, so that the CTAs running at
+  // the same time gather from the same head's K/V and share it in L2 (the
+  // vertical/slash lists of long sequences; for full causal rows the
+  // across-head order balances better)
+  int head_major;
   float scale, scale_log2;
   void* o;
   int64_t osb, oss, osh;
@@ -217,8 +223,9 @@ __device__ __forceinline__ void pf_set_range(uint32_t* bm, int t0, int t1) {
 // Build the schedule of unit u (whole warp 0).
 __device__ void pf_build_sched(const PrefillParams& p, int u, PfSched& sc, int lane) {
   const int per_sg = p.B * p.Hkv * p.n_hgrp;
-  const int sg = p.n_subgrp - 1 - u / per_sg;  // heaviest (latest rows) first
-  const int rest = u % per_sg;
+  const int sg = p.head_major ? p.n_subgrp - 1 - u % p.n_subgrp
+                              : p.n_subgrp - 1 - u / per_sg;  // heaviest (latest rows) first
+  const int rest = p.head_major ? u / p.n_subgrp : u % per_sg;
   const int hgrp = rest % p.n_hgrp;
   const int bg = rest / p.n_hgrp;
   const int g = bg % p.Hkv, b = bg / p.Hkv;
