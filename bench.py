@@ -399,7 +399,7 @@ def bench_nsa(torch, sb, dist, args, flush, peaks, peak_kind):
     flops = 4 * 128 * pairs
     ms, _ = time_device(torch, dist, step, max(3, args.steps // 10), args.warmup, flush)
     tf = flops / (ms * 1e-3) / 1e12
-    part_bytes = total * H * 16 * (128 + 1) * 4
+    acc_bytes = total * H * (128 + 2) * 4
     cu_txt = ", ".join(str(int(x)) for x in wl.meta["cu_seqlens"])
     res = {"workload": f"NSA selected attention, varlen cu_seqlens [{cu_txt}], Hq=Hkv=4, "
                         "D=128, bf16, top-16 blocks of 64 (block 0, 2 local, 13 random)",
@@ -407,9 +407,11 @@ def bench_nsa(torch, sb, dist, args, flush, peaks, peak_kind):
             "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "roofline": tensor_roofline(flops, ms, peaks, peak_kind, "nsa_main_kernel",
                                         launches=7),
-            "partials_bytes": part_bytes,
-            "note": "block-major: per-(token, head, slot) fp32 partials written and re-read "
-                    "by the combine; six kernels and a memset per step (index build, unit table, main, combine)"}
+            "accumulator_bytes": acc_bytes,
+            "note": "block-major in two passes over the units (row maxima, then exp2(S - M) V "
+                    "added into an fp32 [token, head, 128] accumulator at L2); seven kernels and "
+                    "two memsets per step (index count/scan/fill, unit table, pass 1, pass 2, "
+                    "finalize)"}
     if not args.no_cpu_baseline and dist.rank == 0:
         try:
             res["oracle"] = oracle_sample_nsa(wl, flops)

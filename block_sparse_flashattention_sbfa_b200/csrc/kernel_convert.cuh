@@ -136,11 +136,6 @@ __global__ void __launch_bounds__(kCvThreads)
 // ----------------------------------------------------------------------------
 constexpr int kCalThreads = 256;
 
-__device__ __forceinline__ uint32_t cal_key(float v) {
-  const uint32_t u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 __global__ void __launch_bounds__(kCalThreads) calibrate_kernel(const float* __restrict__ smax,
                                                                 int n_qb, int k_top,
                                                                 float* __restrict__ T) {
@@ -160,7 +155,7 @@ __global__ void __launch_bounds__(kCalThreads) calibrate_kernel(const float* __r
     for (int b = threadIdx.x; b < 256; b += kCalThreads) hist[b] = 0;
     __syncthreads();
     for (int j = threadIdx.x; j < i; j += kCalThreads) {
-      const uint32_t u = cal_key(cand[j]);
+      const uint32_t u = f32_order_key(cand[j]);
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
     }
     __syncthreads();
@@ -179,10 +174,7 @@ __global__ void __launch_bounds__(kCalThreads) calibrate_kernel(const float* __r
     mask |= 255u << shift;
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    const uint32_t u = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
-    T[row] = __uint_as_float(u);
-  }
+  if (threadIdx.x == 0) T[row] = f32_from_order_key(prefix);
 }
 
 }  // namespace sbfa

@@ -14,17 +14,31 @@
 //   2. nsa_units_kernel flattens the units: one unit = one key block and up
 //      to 128 query rows (entries x G query heads) that selected it; the
 //      table row of unit u holds its key rows, list entries and kv head.
-//   3. nsa_main_kernel: every CTA takes a contiguous range of units (units
-//      of one key block are adjacent, so neighbouring CTAs share K/V tiles
-//      in L2).  Q rows are gathered four at a time by TMA (tile::gather4
-//      over a (token x head) row map) into a 128B-swizzled tile, K/V come by
-//      TMA, S = Q K^T and O = P V run on tcgen05 with fp32 accumulators in
-//      TMEM.  Each row's result over that one block is an fp32 partial
-//      (o, lse) stored at its (token, head, slot); the epilogue stages each
-//      warp's rows in shared memory so that stores write whole 128-byte rows.
-//   4. nsa_combine_kernel merges the top-k partials of every (token, head)
-//      with the LSE combine.
+//   3. nsa_main_kernel<1> (row maxima): every CTA takes its share of the
+//      units (chunks of kNsaChunk consecutive units dealt out round-robin,
+//      so that the whole grid sweeps the sorted (kv head, sequence, block)
+//      order together).  Q rows are gathered four at a time by TMA
+//      (tile::gather4 over a (token x head) row map) into a 128B-swizzled
+//      tile, K comes by TMA, S = Q K^T runs on tcgen05 into TMEM, and each
+//      row's largest visible score over the block (log2 domain) is merged
+//      into M[row] with an integer atomic max on an order-preserving key.
+//   4. nsa_main_kernel<2> (accumulation): the same units again.  With M[row]
+//      the maximum over all of the row's selected keys, P = exp2(S - M) <= 1
+//      needs no rescaling between blocks: O = P V runs on tcgen05 and each
+//      row's unnormalised O and sum of P are added into an fp32 accumulator
+//      [token, head, 128] and l[token, head] by red.global.add, staged so
+//      that every reduction instruction covers whole 128-byte row pieces.
+//      The sweep order keeps the accumulator rows of the current (kv head,
+//      sequence) in L2, so the adds do not go to DRAM.
+//   5. nsa_finalize_kernel: o = acc / l in bf16, lse = ln 2 (M + log2 l).
+//
+// The sum over a row's blocks is the LSE combine of its per-block results
+// with every term scaled by exp2(-M) up front; the additions into the
+// accumulator happen in no fixed order, so results can differ between runs
+// in the last bits of the fp32 sums (never by more than fp32 rounding).
 #pragma once
+
+#include <type_traits>
 
 #include "sbfa_ptx.cuh"
 
@@ -47,8 +61,9 @@ struct NsaParams {
   int2* unit_b;        // [max units] {sequence start, sequence end}
   int max_units;
   int hist_tokens;     // tokens per CTA of the shared-memory histogram kernels
-  float* part_o;       // [total * Hq * topk, 128]
-  float* part_lse;     // [total * Hq * topk]
+  float* acc;          // [total * Hq, 128] unnormalised O, zeroed before pass 2
+  float* l_acc;        // [total * Hq] sum of P, zeroed before pass 2
+  uint32_t* m_key;     // [total * Hq] order key of M (log2 domain), zeroed before pass 1
   __nv_bfloat16* o;
   int64_t oss, osh;
   float* lse;          // [Hq, total]
@@ -220,24 +235,38 @@ __global__ void __launch_bounds__(kNsaIdxThreads) nsa_fill_kernel(NsaParams p) {
   }
 }
 
+
 // ----------------------------------------------------------------------------
-// main kernel
+// main kernel (two passes over the same units)
 // ----------------------------------------------------------------------------
 constexpr int kNsaThreads = 384;
+constexpr int kNsaChunk = 4;  // consecutive units a CTA takes at a time
 
-struct NsaSmem {
-  alignas(1024) uint8_t q[2][kQTileBytes];
-  alignas(1024) uint8_t k[2][kTileBytes];
-  alignas(1024) uint8_t v[2][kTileBytes];
-  alignas(1024) uint8_t p[2][kPTileBytes];
+// Pass 1 keeps four units in flight (Q and K only); pass 2 two (Q, K, V, P).
+struct NsaSmem1 {
+  static constexpr int NS = 4;
+  alignas(1024) uint8_t q[NS][kQTileBytes];
+  alignas(1024) uint8_t k[NS][kTileBytes];
+  uint32_t tmem_base;
+  int abort_flag;
+  uint64_t k_full[NS], q_full[NS][2];  // q_full[stage][producer warp]
+  uint64_t s_full[NS], p_full[NS];     // p_full: the warpgroup has read S
+  uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
+};
+struct NsaSmem2 {
+  static constexpr int NS = 2;
+  alignas(1024) uint8_t q[NS][kQTileBytes];
+  alignas(1024) uint8_t k[NS][kTileBytes];
+  alignas(1024) uint8_t v[NS][kTileBytes];
+  alignas(1024) uint8_t p[NS][kPTileBytes];
   // epilogue staging: each softmax warp turns its 32 rows x 32 fp32 columns
-  // around here so that every store instruction writes whole 128-byte rows
+  // around here so that every reduction instruction covers 128-byte row pieces
   alignas(16) float stage[8][32][32];
   uint32_t tmem_base;
   int abort_flag;
-  uint64_t k_full[2], v_full[2], q_full[2][2];  // q_full[buffer][producer warp]
-  uint64_t s_full[2], p_full[2], o_full[2];
-  uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
+  uint64_t k_full[NS], v_full[NS], q_full[NS][2];
+  uint64_t s_full[NS], p_full[NS], o_full[NS];
+  uint64_t mma_drain;
 };
 
 struct NsaUnit {
@@ -279,27 +308,50 @@ __device__ __forceinline__ NsaUnit nsa_unit(const NsaParams& p, int u) {
   return r;
 }
 
+// This CTA's n-th unit and its number of units: chunks of kNsaChunk
+// consecutive units, dealt out round-robin over the CTAs.
+__device__ __forceinline__ int nsa_cta_unit(int n) {
+  return (n / kNsaChunk) * kNsaChunk * static_cast<int>(gridDim.x) +
+         static_cast<int>(blockIdx.x) * kNsaChunk + n % kNsaChunk;
+}
+__device__ __forceinline__ int nsa_cta_units(int n_all) {
+  const int per_round = kNsaChunk * static_cast<int>(gridDim.x);
+  const int rounds = n_all / per_round;
+  const int rem = n_all - rounds * per_round;
+  return rounds * kNsaChunk +
+         min(max(rem - static_cast<int>(blockIdx.x) * kNsaChunk, 0), kNsaChunk);
+}
+
+// PASS 1: row maxima of S into m_key.  PASS 2: O = exp2(S - M) V and the
+// sums of P added into acc / l_acc.  Unit n of this CTA uses stage n % NS of
+// the rings; its barriers complete phase (n / NS) & 1.
+template <int PASS>
 __global__ void __launch_bounds__(kNsaThreads, 1)
     nsa_main_kernel(const __grid_constant__ CUtensorMap mapQ,
                     const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const NsaParams p) {
+  using Smem = std::conditional_t<PASS == 1, NsaSmem1, NsaSmem2>;
+  constexpr int NS = Smem::NS;
+  // TMEM columns of stage st: pass 1 S (64); pass 2 S (64, P never goes
+  // there) then O (128) at +128
+  constexpr int kStageCols = PASS == 1 ? 64 : 256;
   extern __shared__ uint8_t smem_raw[];
-  NsaSmem& sm = *reinterpret_cast<NsaSmem*>(
+  Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_all = min(__ldg(p.unit_prefix + p.Hkv * p.nseq * p.nbps), p.max_units);
-  // this CTA's units: the contiguous range [u_lo, u_lo + n_mine)
-  const int u_lo = static_cast<int>(static_cast<int64_t>(n_all) * blockIdx.x / gridDim.x);
-  const int n_mine = static_cast<int>(static_cast<int64_t>(n_all) * (blockIdx.x + 1) / gridDim.x) - u_lo;
+  const int n_mine = nsa_cta_units(n_all);
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NS; ++b) {
       mbar_init(&sm.k_full[b], 1);
-      mbar_init(&sm.v_full[b], 1);
       mbar_init(&sm.q_full[b][0], 1);  // each producer warp arms its own half
       mbar_init(&sm.q_full[b][1], 1);
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.p_full[b], 128);
-      mbar_init(&sm.o_full[b], 1);
+      if constexpr (PASS == 2) {
+        mbar_init(&sm.v_full[b], 1);
+        mbar_init(&sm.o_full[b], 1);
+      }
     }
     mbar_init(&sm.mma_drain, 1);
     sm.abort_flag = 0;
@@ -332,28 +384,29 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     NsaUnit cur{}, nxt{};
     int c0 = -1, c1 = -1, n0 = -1, n1 = -1, first = 0, first_n = 0;
     if (n_mine > 0) {
-      cur = nsa_unit(p, u_lo);
+      cur = nsa_unit(p, nsa_cta_unit(0));
       load_codes(cur, c0, c1);
       first = __ldg(p.list + cur.e0);
     }
-    if (n_mine > 1) nxt = nsa_unit(p, u_lo + 1);
+    if (n_mine > 1) nxt = nsa_unit(p, nsa_cta_unit(1));
     bool ok = true;
     // last unit whose Q (and, for warp 0, K) / V copies this warp issued into
-    // each buffer, for the drain before exit; a buffer is refilled only after
+    // each stage, for the drain before exit; a stage is refilled only after
     // its previous contents were consumed, so only that last phase can pend
-    int qk_last[2] = {-1, -1}, v_last[2] = {-1, -1};
-    // Buffers of unit n (index n & 1) were last used by unit n - 2: Q and K
-    // are free once QK(n - 2) has completed (s_full), V once PV(n - 2) has
-    // (o_full), which comes after QK(n - 1) and so after Q(n - 1) landed.
+    int qk_last[NS], v_last[NS];
+#pragma unroll
+    for (int b = 0; b < NS; ++b) qk_last[b] = v_last[b] = -1;
+    // Stage n % NS was last used by unit n - NS: Q and K are free once
+    // QK(n - NS) has completed (s_full), V once PV(n - NS) has (o_full).
     for (int n = 0; n < n_mine && ok; ++n) {
-      const int b = n & 1;
-      const uint32_t pw = ((n >> 1) & 1) ^ 1u;
+      const int b = n % NS;
+      const uint32_t pw = ((n / NS) & 1) ^ 1u;
       if (n + 1 < n_mine) {
         load_codes(nxt, n0, n1);
         first_n = __ldg(p.list + nxt.e0);
       }
       NsaUnit nn{};
-      if (n + 2 < n_mine) nn = nsa_unit(p, u_lo + n + 2);
+      if (n + 2 < n_mine) nn = nsa_unit(p, nsa_cta_unit(n + 2));
       if (lane == 0) ok = mbar_wait(&sm.s_full[b], pw, wctx);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
@@ -383,17 +436,19 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         tma_gather4_2d(sm.q[b] + colh * 16384 + (half * 64 + rl) * 128, &mapQ,
                        &sm.q_full[b][half], colh * 64, y[0], y[1], y[2], y[3]);
       }
-      if (half == 0) {
-        if (lane == 0) {
-          ok = mbar_wait(&sm.o_full[b], pw, wctx);
-          if (ok) {
-            v_last[b] = n;
-            mbar_arrive_expect_tx(&sm.v_full[b], kTileBytes);
-            tma_load_4d(sm.v[b], &mapV, &sm.v_full[b], 0, cur.g, cur.key0, 0);
-            tma_load_4d(sm.v[b] + 8192, &mapV, &sm.v_full[b], 64, cur.g, cur.key0, 0);
+      if constexpr (PASS == 2) {
+        if (half == 0) {
+          if (lane == 0) {
+            ok = mbar_wait(&sm.o_full[b], pw, wctx);
+            if (ok) {
+              v_last[b] = n;
+              mbar_arrive_expect_tx(&sm.v_full[b], kTileBytes);
+              tma_load_4d(sm.v[b], &mapV, &sm.v_full[b], 0, cur.g, cur.key0, 0);
+              tma_load_4d(sm.v[b] + 8192, &mapV, &sm.v_full[b], 64, cur.g, cur.key0, 0);
+            }
           }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
       cur = nxt; nxt = nn;
       c0 = n0; c1 = n1; first = first_n;
@@ -401,30 +456,31 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     // no copy may still be landing in shared memory when the CTA exits
     __syncwarp();
     if (lane == 0) {
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < NS; ++b) {
         if (qk_last[b] >= 0) {
-          const uint32_t ph = (qk_last[b] >> 1) & 1;
+          const uint32_t ph = (qk_last[b] / NS) & 1;
           mbar_wait_short(&sm.q_full[b][half], ph);
           if (half == 0) mbar_wait_short(&sm.k_full[b], ph);
         }
-        if (half == 0 && v_last[b] >= 0) mbar_wait_short(&sm.v_full[b], (v_last[b] >> 1) & 1);
+        if constexpr (PASS == 2)
+          if (half == 0 && v_last[b] >= 0) mbar_wait_short(&sm.v_full[b], (v_last[b] / NS) & 1);
       }
     }
   } else if (warp == 1) {
     // ===================== MMA issuer =====================
-    // Order: QK(0), QK(1), PV(0), QK(2), PV(1), ... so that the softmax of
-    // one unit overlaps the QK of the next.
+    // Pass 2 order: QK(0), QK(1), PV(0), QK(2), PV(1), ... so that the softmax
+    // of one unit overlaps the QK of the next; S(n + 1) reuses the columns of
+    // S(n - 1), whose P was consumed by PV(n - 1), issued before it.  Pass 1
+    // has no PV: QK(n) waits until the warpgroup has read S(n - NS).
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0);
-      const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
       const uint64_t qdesc0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
-      const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.v[0]), 8192, 1024);
-      const uint64_t pdesc0 = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
       bool ok = true;
       auto issue_qk = [&](int n) -> bool {
-        const int b = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
+        const int b = n % NS;
+        const uint32_t ph = (n / NS) & 1;
+        if (PASS == 1 && n >= NS && !mbar_wait(&sm.p_full[b], ph ^ 1u, wctx)) return false;
         if (!mbar_wait(&sm.q_full[b][0], ph, wctx) || !mbar_wait(&sm.q_full[b][1], ph, wctx) ||
             !mbar_wait(&sm.k_full[b], ph, wctx))
           return false;
@@ -435,30 +491,37 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off_q = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
           const uint32_t off_k = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + b * 256, qd + off_q, kd + off_k, idesc_qk, kk ? 1u : 0u);
+          umma_ss(tmem + b * kStageCols, qd + off_q, kd + off_k, idesc_qk, kk ? 1u : 0u);
         }
         umma_commit(&sm.s_full[b]);
         return true;
       };
-      auto issue_pv = [&](int n) -> bool {
-        const int b = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        if (!mbar_wait(&sm.p_full[b], ph, wctx) || !mbar_wait(&sm.v_full[b], ph, wctx))
-          return false;
-        tc_fence_after();
-        const uint64_t pd = pdesc0 + (b * kPTileBytes >> 4);
-        const uint64_t vd = vdesc0 + (b * kTileBytes >> 4);
+      if constexpr (PASS == 1) {
+        for (int n = 0; n < n_mine && ok; ++n) ok = issue_qk(n);
+      } else {
+        const uint32_t idesc_pv = idesc_bf16(128, 128, 1);
+        const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.v[0]), 8192, 1024);
+        const uint64_t pdesc0 = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
+        auto issue_pv = [&](int n) -> bool {
+          const int b = n % NS;
+          const uint32_t ph = (n / NS) & 1;
+          if (!mbar_wait(&sm.p_full[b], ph, wctx) || !mbar_wait(&sm.v_full[b], ph, wctx))
+            return false;
+          tc_fence_after();
+          const uint64_t pd = pdesc0 + (b * kPTileBytes >> 4);
+          const uint64_t vd = vdesc0 + (b * kTileBytes >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_ss(tmem + b * 256 + 128, pd + (kk * 32 >> 4), vd + (kk * 2048 >> 4), idesc_pv,
-                  kk ? 1u : 0u);
-        umma_commit(&sm.o_full[b]);
-        return true;
-      };
-      if (n_mine > 0) ok = issue_qk(0);
-      for (int n = 0; n < n_mine && ok; ++n) {
-        if (n + 1 < n_mine) ok = issue_qk(n + 1);
-        if (ok) ok = issue_pv(n);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(tmem + b * kStageCols + 128, pd + (kk * 32 >> 4), vd + (kk * 2048 >> 4),
+                    idesc_pv, kk ? 1u : 0u);
+          umma_commit(&sm.o_full[b]);
+          return true;
+        };
+        if (n_mine > 0) ok = issue_qk(0);
+        for (int n = 0; n < n_mine && ok; ++n) {
+          if (n + 1 < n_mine) ok = issue_qk(n + 1);
+          if (ok) ok = issue_pv(n);
+        }
       }
       // drain every tcgen05 op before TMEM is released: a commit to a barrier
       // nothing else uses completes its single phase only then
@@ -468,107 +531,122 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ===================== softmax / epilogue warpgroups (ping-pong) =====================
-    const int b = (warp - 4) >> 2;
-    const int r = tid - 128 - 128 * b;
+    const int wg = (warp - 4) >> 2;  // units n = wg, wg + 2, ...
+    const int r = tid - 128 - 128 * wg;
     const int quarter = warp & 3;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * 256;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float NEG = -INFINITY;
     bool ok = true;
-    // this warpgroup's units n = b, b + 2, ...: row codes one unit ahead
+    // row codes (and, in pass 2, the row's M) one unit ahead
     NsaUnit un_next{};
     int code_next = -1;
-    if (b < n_mine) {
-      un_next = nsa_unit(p, u_lo + b);
+    uint32_t mkey_next = 0;
+    auto row_of = [&](const NsaUnit& un, int code) -> int64_t {
+      return static_cast<int64_t>(code / p.topk) * p.Hq + un.g * p.G + r % p.G;
+    };
+    auto fetch = [&](int n) {
+      un_next = nsa_unit(p, nsa_cta_unit(n));
       code_next = r / p.G < un_next.ne ? __ldg(p.list + un_next.e0 + r / p.G) : -1;
-    }
-    for (int n = b; n < n_mine && ok; n += 2) {
-      const uint32_t ph = (n >> 1) & 1;
+      if (PASS == 2 && code_next >= 0) mkey_next = p.m_key[row_of(un_next, code_next)];
+    };
+    if (wg < n_mine) fetch(wg);
+    for (int n = wg; n < n_mine && ok; n += 2) {
+      const int st = n % NS;
+      const uint32_t ph = (n / NS) & 1;
+      const uint32_t lane_addr = lane_base + st * kStageCols;
       const NsaUnit un = un_next;
       const int code = code_next;
-      if (n + 2 < n_mine) {
-        un_next = nsa_unit(p, u_lo + n + 2);
-        code_next = r / p.G < un_next.ne ? __ldg(p.list + un_next.e0 + r / p.G) : -1;
-      }
+      const uint32_t mkey = mkey_next;
+      if (n + 2 < n_mine) fetch(n + 2);
       const bool valid = code >= 0;
-      int t = 0, slot = 0, tl = 0, L = 0;
+      int tl = 0, L = 0;
+      int64_t row = -1;
       if (valid) {
-        t = code / p.topk;
-        slot = code % p.topk;
-        tl = t - un.base;
+        row = row_of(un, code);
+        tl = code / p.topk - un.base;
         L = un.end - un.base;
       }
       // tcgen05.ld is warp-collective: the warp agrees before leaving
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], ph, wctx))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[st], ph, wctx))) { ok = false; break; }
       tc_fence_after();
       float s[64];
       tmem_ld32(lane_addr, s);
       tmem_ld32(lane_addr + 32, s + 32);
-      float mx = NEG;
       const int kb = un.key0 - un.base;  // first key of the block, sequence-local
       if (__all_sync(0xffffffffu, valid && kb + 63 < L && (!p.causal || kb + 63 <= tl))) {
         // every key of the block is visible to every row of this warp
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          s[c] *= p.scale_log2;
-          mx = fmaxf(mx, s[c]);
-        }
+        for (int c = 0; c < 64; ++c) s[c] *= p.scale_log2;
       } else {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int key = kb + c;
           const bool vis = valid && key < L && (!p.causal || key <= tl);
           s[c] = vis ? s[c] * p.scale_log2 : NEG;
-          mx = fmaxf(mx, s[c]);
         }
       }
-      const float mu = (mx == NEG) ? 0.f : mx;
-      float l = 0.f;
-      uint32_t pk[32];
+      if constexpr (PASS == 1) {
+        // S is in registers: the MMA warp may overwrite its columns
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[st]);
+        float m4[4] = {NEG, NEG, NEG, NEG};
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2_approx(s[c] - mu), p1 = ex2_approx(s[c + 1] - mu);
-        l += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-      }
-      const uint32_t prow = smem_u32(sm.p[b]);
+        for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], s[c], s[c + 1]);
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        if (valid && mx > NEG) atomicMax(p.m_key + row, f32_order_key(mx));
+      } else {
+        // ---- P = exp2(S - M) with M the row's maximum over all its blocks
+        const float M = f32_from_order_key(mkey);
+        const float mu = (M > NEG && M < INFINITY) ? M : 0.f;  // no visible key: key 0 (NaN)
+        float l = 0.f;
+        uint32_t pk[32];
+        {
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, cc)),
-                     "r"(pk[cc * 4]), "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]), "r"(pk[cc * 4 + 3])
-                     : "memory");
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&sm.p_full[b]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[b], ph, wctx))) { ok = false; break; }
-      tc_fence_after();
-      const int h = un.g * p.G + r % p.G;
-      const int64_t prow_idx = (static_cast<int64_t>(t) * p.Hq + h) * p.topk + slot;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      // 32 columns at a time: each lane parks its row in the warp's staging
-      // tile (16-byte pieces rotated by row to spread the banks), then lane
-      // group i / 8 of each store writes the 128 contiguous bytes of one row
-      float (*stg)[32] = sm.stage[warp - 4];
-      float ob[32];
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2_approx(s[c] - mu), p1 = ex2_approx(s[c + 1] - mu);
+            const int a = ((c >> 1) & 1) * 2;
+            add2(l4[a], l4[a + 1], p0, p1);
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        }
+        const uint32_t prow = smem_u32(sm.p[st]);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, cc)),
+                       "r"(pk[cc * 4]), "r"(pk[cc * 4 + 1]), "r"(pk[cc * 4 + 2]),
+                       "r"(pk[cc * 4 + 3])
+                       : "memory");
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[st]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[st], ph, wctx))) { ok = false; break; }
+        tc_fence_after();
+        // 32 columns at a time: each lane parks its row in the warp's staging
+        // tile (16-byte pieces rotated by row to spread the banks), then lane
+        // group i / 8 of each reduction covers the 128 contiguous bytes of one row
+        float (*stg)[32] = sm.stage[warp - 4];
+        float ob[32];
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(lane_addr + 128 + c * 32, ob);
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(lane_addr + 128 + c * 32, ob);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          *reinterpret_cast<float4*>(&stg[lane][4 * (i ^ (lane & 7))]) =
-              make_float4(ob[4 * i] * inv, ob[4 * i + 1] * inv, ob[4 * i + 2] * inv,
-                          ob[4 * i + 3] * inv);
-        __syncwarp();
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<float4*>(&stg[lane][4 * (i ^ (lane & 7))]) =
+                make_float4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+          __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + (lane >> 3), piece = lane & 7;
-          const long long dst_row = __shfl_sync(0xffffffffu, valid ? prow_idx : -1ll, rr);
-          const float4 x = *reinterpret_cast<const float4*>(&stg[rr][4 * (piece ^ (rr & 7))]);
-          if (dst_row >= 0)
-            *reinterpret_cast<float4*>(p.part_o + dst_row * 128 + c * 32 + 4 * piece) = x;
+          for (int i = 0; i < 8; ++i) {
+            const int rr = 4 * i + (lane >> 3), piece = lane & 7;
+            const long long dst_row = __shfl_sync(0xffffffffu, static_cast<long long>(row), rr);
+            const float4 x = *reinterpret_cast<const float4*>(&stg[rr][4 * (piece ^ (rr & 7))]);
+            if (dst_row >= 0) red_add_v4_f32(p.acc + dst_row * 128 + c * 32 + 4 * piece, x);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        if (valid && l > 0.f) atomicAdd(p.l_acc + row, l);
       }
-      if (valid) p.part_lse[prow_idx] = l > 0.f ? (mu + lg2_approx(l)) * 0.69314718055994531f : NEG;
     }
   }
   tc_fence_before();
@@ -579,84 +657,24 @@ __global__ void __launch_bounds__(kNsaThreads, 1)
   }
 }
 
-// One warp per (token, query head): LSE combine of its valid slots.
-__global__ void nsa_combine_kernel(NsaParams p) {
-  const int64_t wg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wg >= static_cast<int64_t>(p.total) * p.Hq) return;
-  const int t = static_cast<int>(wg / p.Hq), h = static_cast<int>(wg % p.Hq);
-  const int g = h / p.G;
-  const int s = nsa_seq_of(p.cu, p.nseq, t);
-  const int L = p.cu[s + 1] - p.cu[s];
-  const int nb = (L + 63) / 64;
-  const int* sl = p.sel + (static_cast<int64_t>(t) * p.Hkv + g) * p.topk;
-  const int64_t row = (static_cast<int64_t>(t) * p.Hq + h) * p.topk;
-  if (p.topk <= 32) {
-    // lane k holds slot k's lse; the partial rows of the valid slots are
-    // then fetched eight at a time, all loads of a batch in flight together
-    float lv = -INFINITY;
-    if (lane < p.topk) {
-      const int j = __ldg(sl + lane);
-      if (j >= 0 && j < nb) lv = p.part_lse[row + lane];
-    }
-    const float M = warp_max_f32(lv);
-    const float Mn = (M == -INFINITY) ? 0.f : M;
-    const float w = (lv == -INFINITY) ? 0.f : __expf(lv - Mn);
-    float W = w;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
-    unsigned vm = __ballot_sync(0xffffffffu, w > 0.f);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    while (vm) {
-      int ks[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        ks[u] = vm ? __ffs(vm) - 1 : -1;
-        vm &= vm - 1u;
-      }
-      float4 xs[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (ks[u] >= 0)
-          xs[u] = *reinterpret_cast<const float4*>(p.part_o + (row + ks[u]) * 128 + lane * 4);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (ks[u] < 0) continue;
-        const float wu = __shfl_sync(0xffffffffu, w, ks[u]);
-        acc.x += wu * xs[u].x; acc.y += wu * xs[u].y; acc.z += wu * xs[u].z; acc.w += wu * xs[u].w;
-      }
-    }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    __nv_bfloat16* op = p.o + static_cast<int64_t>(t) * p.oss + h * p.osh + lane * 4;
-    reinterpret_cast<__nv_bfloat162*>(op)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    reinterpret_cast<__nv_bfloat162*>(op)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    if (lane == 0) p.lse[static_cast<int64_t>(h) * p.total + t] = W > 0.f ? Mn + __logf(W) : -INFINITY;
-    return;
-  }
-  float M = -INFINITY;
-  for (int k = 0; k < p.topk; ++k) {
-    const int j = __ldg(sl + k);
-    if (j < 0 || j >= nb) continue;
-    M = fmaxf(M, p.part_lse[row + k]);
-  }
-  const float Mn = (M == -INFINITY) ? 0.f : M;
-  float W = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k = 0; k < p.topk; ++k) {
-    const int j = __ldg(sl + k);
-    if (j < 0 || j >= nb) continue;
-    const float lv = p.part_lse[row + k];
-    if (lv == -INFINITY) continue;
-    const float w = __expf(lv - Mn);
-    W += w;
-    const float4 x = *reinterpret_cast<const float4*>(p.part_o + (row + k) * 128 + lane * 4);
-    acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
-  }
-  const float inv = W > 0.f ? 1.f / W : 0.f;
+// One warp per (token, query head), four columns a lane: o = acc / l,
+// lse = ln 2 (M + log2 l).
+__global__ void nsa_finalize_kernel(NsaParams p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = i >> 5;
+  const int lane = static_cast<int>(i & 31);
+  if (row >= static_cast<int64_t>(p.total) * p.Hq) return;
+  const int t = static_cast<int>(row / p.Hq), h = static_cast<int>(row % p.Hq);
+  const float l = p.l_acc[row];
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const float4 x = *reinterpret_cast<const float4*>(p.acc + row * 128 + lane * 4);
   __nv_bfloat16* op = p.o + static_cast<int64_t>(t) * p.oss + h * p.osh + lane * 4;
-  reinterpret_cast<__nv_bfloat162*>(op)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  reinterpret_cast<__nv_bfloat162*>(op)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  if (lane == 0) p.lse[static_cast<int64_t>(h) * p.total + t] = W > 0.f ? Mn + __logf(W) : -INFINITY;
+  reinterpret_cast<__nv_bfloat162*>(op)[0] = __floats2bfloat162_rn(x.x * inv, x.y * inv);
+  reinterpret_cast<__nv_bfloat162*>(op)[1] = __floats2bfloat162_rn(x.z * inv, x.w * inv);
+  if (lane == 0)
+    p.lse[static_cast<int64_t>(h) * p.total + t] =
+        l > 0.f ? (f32_from_order_key(p.m_key[row]) + lg2_approx(l)) * 0.69314718055994531f
+                : -INFINITY;
 }
 
 }  // namespace sbfa

@@ -421,7 +421,8 @@ void set_table(sbfa::PrefillParams& p, const sbfa_table* t, int nmax_override = 
 // NSA selected attention workspace
 // ---------------------------------------------------------------------------
 struct NsaWs {
-  size_t count, cursor, offset, unit_prefix, list, unit_a, unit_b, part_lse, part_o, total;
+  size_t count, cursor, offset, unit_prefix, list, unit_a, unit_b, acc, l_acc, m_key, end_zero,
+      total;
   int64_t max_units;
 };
 
@@ -441,8 +442,11 @@ NsaWs nsa_ws_layout(int nseq, int total, int max_seqlen, int Hq, int Hkv, int to
   w.max_units = static_cast<int64_t>(total) * Hkv * topk / per_unit + static_cast<int64_t>(nb);
   w.unit_a = off; off += al256(static_cast<size_t>(w.max_units) * 16);
   w.unit_b = off; off += al256(static_cast<size_t>(w.max_units) * 8);
-  w.part_lse = off; off += al256(static_cast<size_t>(total) * Hq * topk * 4);
-  w.part_o = off; off += al256(static_cast<size_t>(total) * Hq * topk * 128 * 4);
+  // accumulator, sums of P and row-maximum keys: one span, zeroed per call
+  w.acc = off; off += al256(static_cast<size_t>(total) * Hq * 128 * 4);
+  w.l_acc = off; off += al256(static_cast<size_t>(total) * Hq * 4);
+  w.m_key = off; off += al256(static_cast<size_t>(total) * Hq * 4);
+  w.end_zero = off;
   w.total = off;
   return w;
 }
@@ -958,8 +962,9 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   p.unit_b = reinterpret_cast<int2*>(w + L.unit_b);
   if (L.max_units >= (1ll << 31)) return fail(SBFA_ERR_UNSUPPORTED, "too many units");
   p.max_units = static_cast<int>(L.max_units);
-  p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
-  p.part_o = reinterpret_cast<float*>(w + L.part_o);
+  p.acc = reinterpret_cast<float*>(w + L.acc);
+  p.l_acc = reinterpret_cast<float*>(w + L.l_acc);
+  p.m_key = reinterpret_cast<uint32_t*>(w + L.m_key);
   p.o = static_cast<__nv_bfloat16*>(o.ptr); p.oss = o.ss; p.osh = o.sh;
   p.lse = lse;
   p.status = status;
@@ -971,6 +976,7 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   SBFA_TRY(encode_bshd(&mk, k, 1, total, Hkv, 64));
   SBFA_TRY(encode_bshd(&mv, v, 1, total, Hkv, 64));
   SBFA_CUDA(cudaMemsetAsync(p.count, 0, nb * 4, st));
+  SBFA_CUDA(cudaMemsetAsync(w + L.acc, 0, L.end_zero - L.acc, st));
   // inverted index: shared-memory histograms when the key space fits, else
   // one global atomic per (warp, key)
   const bool hist = nb <= sbfa::kNsaHistMaxKeys;
@@ -1000,19 +1006,25 @@ sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, in
   SBFA_CUDA(cudaGetLastError());
   sbfa::nsa_units_kernel<<<static_cast<unsigned>((L.max_units + 255) / 256), 256, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
-  const size_t smem = sizeof(sbfa::NsaSmem) + 1024;
+  const size_t smem1 = sizeof(sbfa::NsaSmem1) + 1024;
+  const size_t smem2 = sizeof(sbfa::NsaSmem2) + 1024;
   static bool attr_set[64] = {false};
   int dev = 0;
   SBFA_CUDA(cudaGetDevice(&dev));
   if (!attr_set[dev]) {
-    SBFA_CUDA(cudaFuncSetAttribute(sbfa::nsa_main_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::nsa_main_kernel<1>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1));
+    SBFA_CUDA(cudaFuncSetAttribute(sbfa::nsa_main_kernel<2>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2));
     attr_set[dev] = true;
   }
-  sbfa::nsa_main_kernel<<<di.sms, sbfa::kNsaThreads, smem, st>>>(mq, mk, mv, p);
+  // pass 1: row maxima; pass 2: accumulation over the same units
+  sbfa::nsa_main_kernel<1><<<di.sms, sbfa::kNsaThreads, smem1, st>>>(mq, mk, mv, p);
+  SBFA_CUDA(cudaGetLastError());
+  sbfa::nsa_main_kernel<2><<<di.sms, sbfa::kNsaThreads, smem2, st>>>(mq, mk, mv, p);
   SBFA_CUDA(cudaGetLastError());
   const int64_t rows = static_cast<int64_t>(total) * Hq;
-  sbfa::nsa_combine_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);
+  sbfa::nsa_finalize_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);
   SBFA_CUDA(cudaGetLastError());
   return SBFA_OK;
 }

@@ -398,6 +398,13 @@ __device__ __forceinline__ void mul2(float& a0, float& a1, float b) {
       : "f"(b));
 }
 // max of three floats in one instruction (sm_100 three-input FMNMX)
+// Fire-and-forget fp32 add of four consecutive floats (16-byte aligned),
+// performed at L2.
+__device__ __forceinline__ void red_add_v4_f32(float* addr, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -413,6 +420,16 @@ __device__ __forceinline__ float warp_max_f32(float v) {
   u = __reduce_max_sync(0xffffffffu, u);
   u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
   return __uint_as_float(u);
+}
+// Order-preserving 32-bit key of a float: a < b (as floats, -0 < +0) iff
+// key(a) < key(b) (as unsigned), so that integer max / radix selection works
+// on floats.  Key 0 is below every float's key; its inverse is a NaN.
+__device__ __forceinline__ uint32_t f32_order_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float f32_from_order_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;

@@ -360,10 +360,13 @@ sbfa_status sbfa_fwd_vertical_slash_varlen(
  * ignored); o like q; lse: fp32 [Hq, total].  sel: int32 [total, Hkv, topk]
  * contiguous.  block must be 64; Hq/Hkv must divide 128.  ws: device
  * workspace of sbfa_varlen_selected_workspace_size() bytes (contents need
- * no initialisation).  Runs on `stream`: a memset and the inverted-index
- * count / scan / fill, the unit table, the block-major tcgen05 kernel that
- * writes one fp32 partial (o, lse) per (token, head, slot), and the LSE
- * combine of each row's partials.
+ * no initialisation).  Runs on `stream`: two memsets, the inverted-index
+ * count / scan / fill, the unit table, and two block-major tcgen05 passes
+ * over the (key block, query rows) units: the first takes each row's
+ * largest score M, the second adds exp2(S - M) V and the sums of
+ * exp2(S - M) into an fp32 accumulator per (token, head); a last kernel
+ * writes o = accumulator / sum and lse.  The additions happen in no fixed
+ * order: results can differ between runs within fp32 rounding.
  */
 sbfa_status sbfa_fwd_varlen_selected(const int32_t* cu_seqlens, int32_t nseq, int32_t total,
                                      int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t D,
