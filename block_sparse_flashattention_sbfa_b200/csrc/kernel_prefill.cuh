@@ -923,60 +923,57 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
           }
         };
-        float rm[2] = {NEG, NEG};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float sh[64];
-          tmem_ld64(lane_addr + 64 * h, sh);
-          mask_half(sh, h);
-          float m4[4] = {NEG, NEG, NEG, NEG};
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], sh[c], sh[c + 1]);
-          rm[h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        }
+        // ---- one pass per 64-key half: mask, row max, P = exp2(s - m) into
+        // TMEM as bf16 pairs over the first 64 columns of S (half 0 -> columns
+        // 0..31, half 1 -> 32..63; half 1 is read from columns 64..127, which
+        // P never overwrites).  The running max m is raised (lazily: only past
+        // 2^8) from each half's max as it comes; if half 1 raises it, half 0's
+        // P, already in TMEM, is scaled to the new m (rare after a row's first
+        // tiles).  O and l of earlier tiles take the product of the factors.
         const int my_keep = segm;
         const int flag = tmask;
-        // ---- online softmax over the kept halves (log2 domain, lazy rescale)
-        float rmax = NEG;
-        if (my_keep & 1) rmax = rm[0];
-        if (my_keep & 2) rmax = fmaxf(rmax, rm[1]);
-        float alpha = 1.f;
-        bool resc = false;
-        if (rmax != NEG) {
-          const float mrow = rmax * p.scale_log2;
-          if (mrow > m_used + 8.f) {
-            alpha = ex2_approx(m_used - mrow);
-            resc = true;
-            m_used = mrow;
-          }
-        }
-        const float mu = (m_used == NEG) ? 0.f : m_used;
-        // the commit behind s_full also covers the previous PV: O is stable here
-        if (npv > 0 && __any_sync(0xffffffffu, resc)) {
-          pacc[6] += 1;
-          float ob[32];
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32(lane_addr + 128 + c * 32, ob);
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], alpha);
-            tmem_st32(lane_addr + 128 + c * 32, ob);
-          }
-        }
-        // ---- pass 2: P = exp2(s - m) per half, stored as bf16 pairs over the
-        // first 64 columns of S (half 0 -> columns 0..31, half 1 -> 32..63;
-        // half 1 is reloaded from columns 64..127, which P never overwrites)
-        float psum = 0.f;
+        float alpha = 1.f, psum = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
           const bool mine = (my_keep >> h) & 1;
-          // tcgen05.ld is warp-collective: reload when any lane of the warp
-          // keeps this half (rows differ in validity inside a ragged block)
+          // tcgen05.ld is warp-collective: load when any lane of the warp keeps
+          // this half (rows differ in validity inside a ragged block)
           if (__any_sync(0xffffffffu, mine)) {
             float sh[64];
             tmem_ld64(lane_addr + 64 * h, sh);
             mask_half(sh, h);
+            float a_h = 1.f;
+            if (mine) {
+              float m4[4] = {NEG, NEG, NEG, NEG};
+#pragma unroll
+              for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = max3(m4[(c >> 1) & 3], sh[c], sh[c + 1]);
+              const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+              if (mx != NEG) {
+                const float mrow = mx * p.scale_log2;
+                if (mrow > m_used + 8.f) {
+                  a_h = ex2_approx(m_used - mrow);  // 0 while m_used = -inf
+                  m_used = mrow;
+                }
+              }
+            }
+            if (h == 1 && __any_sync(0xffffffffu, a_h != 1.f)) {
+              pacc[4] += 1;
+              tmem_wait_st();
+              float pf[32];
+              tmem_ld32(lane_addr, pf);
+              uint32_t* pu = reinterpret_cast<uint32_t*>(pf);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const float lo = __uint_as_float(pu[c] << 16) * a_h;
+                const float hi = __uint_as_float(pu[c] & 0xffff0000u) * a_h;
+                pu[c] = pack_bf16x2(lo, hi);
+              }
+              tmem_st32_nowait(lane_addr, pf);
+              psum *= a_h;
+            }
+            alpha *= a_h;
+            const float mu = (m_used == NEG) ? 0.f : m_used;
             const float base = mine ? mu : INFINITY;  // exp2(-inf) = 0 for lanes without it
             float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -993,7 +990,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) pk[c] = 0u;
           }
-          tmem_st32(lane_addr + 32 * h, reinterpret_cast<const float*>(pk));
+          if (h == 0) tmem_st32_nowait(lane_addr, reinterpret_cast<const float*>(pk));
+          else tmem_st32(lane_addr + 32, reinterpret_cast<const float*>(pk));
+        }
+        // the commit behind s_full also covers the previous PV: O is stable here
+        if (npv > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          pacc[6] += 1;
+          float ob[32];
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(lane_addr + 128 + c * 32, ob);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], alpha);
+            tmem_st32(lane_addr + 128 + c * 32, ob);
+          }
         }
         l = l * alpha + psum;
         tc_fence_before();
