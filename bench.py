@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 
 import workloads as W  # noqa: E402
 
+DECODE_WORKLOAD = ("speculative+sparse decode B=8 Hq=32 Hkv=8 Lq=1 Lk=32768 D=128 bs=128, "
+                   "dense last 2048 + 32 missed blocks")
 METRIC = ("sparse-attn fwd kept-block TFLOP/s (% bf16 peak); "
           "decode kept-KV GB/s (% HBM)")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -613,9 +615,7 @@ def main():
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(sec_per_step * 1e3, 3), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "speculative+sparse decode B=8 Hq=32 Hkv=8 Lq=1 "
-                                       "Lk=32768 D=128 bs=128, dense last 2048 + 32 missed "
-                                       "blocks", "global_batch": 8, "seq_len": 32768},
+                "config": {"workload": DECODE_WORKLOAD, "global_batch": 8, "seq_len": 32768},
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -664,9 +664,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dec["ms"], 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "speculative+sparse decode B=8 Hq=32 Hkv=8 Lq=1 Lk=32768 "
-                               "D=128 bs=128, dense last 2048 + 32 missed blocks, fused "
-                               "split-KV kernel", "global_batch": 8 * dist.world,
+        "config": {"workload": DECODE_WORKLOAD, "global_batch": 8 * dist.world,
                    "seq_len": 32768, "parallelism": f"replicas x{dist.world}",
                    "l2": "flushed before every step (4x L2 write, then 4x L2 read), outside the timed events"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
