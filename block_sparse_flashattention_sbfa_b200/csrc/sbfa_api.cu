@@ -201,7 +201,7 @@ sbfa_status launch_prefill(sbfa::PrefillParams& p, const sbfa_shape* s, const sb
   p.n_kt = (s->Sk + 63) / 64;
   p.causal = s->causal;
   p.causal_off = s->Sk - s->Sq;
-  p.head_major = p.mode == sbfa::kModeVS ? 1 : 0;
+  p.head_major = (p.mode == sbfa::kModeVS || p.mode == sbfa::kModeGated) ? 1 : 0;
   p.scale = eff_scale(s);
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.k = static_cast<const __nv_bfloat16*>(k.ptr);
