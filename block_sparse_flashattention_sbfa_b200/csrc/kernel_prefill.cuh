@@ -170,6 +170,11 @@ struct PfSmem {
   // epilogue has read O), and only then: a tile with no block in a unit
   // signals nothing, so the phases cannot run ahead of the MMA warp's waits.
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  // split P hand-over (gated): p_full[t] then covers half 0 of tile t's P,
+  // p_full1[t] half 1 (one barrier per half, so that each completes one
+  // phase per key tile and the softmax cannot run one two phases ahead of
+  // the MMA warp's wait); pvh0[t]: the PV of half 0 has completed
+  uint64_t p_full1[2], pvh0[2];
   uint64_t ga_full[2], ga_free[2];  // gate: S^T buffers written / read
   uint64_t kb_done;                 // gate: the unit's keep bitmaps are complete
   uint64_t mma_drain;  // one final commit: every MMA of the CTA has completed
@@ -414,6 +419,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
   constexpr bool gated = MODE == kModeGated;
   constexpr bool has_cols = MODE == kModeVS;
+  // P handed to the MMA warp half by half (half 0's P V then runs while
+  // half 1 is computed): faster where kept blocks are isolated (gated phase
+  // B: 32K 11.9 -> 10.9 ms), slower for full rows, where the extra hand-over
+  // costs more than the overlap gains (dense 16K 2.55 -> 2.73 ms)
+  constexpr bool split_p = gated;
   unsigned long long pacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const long long t_start = clock64();
 
@@ -425,6 +435,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.p_full[i], 128);
       mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.p_full1[i], 128);
+      mbar_init(&sm.pvh0[i], 1);
       mbar_init(&sm.o_free[i], 128);
       mbar_init(&sm.ga_full[i], 1);
       mbar_init(&sm.ga_free[i], 8);  // one arrival per softmax warp
@@ -675,8 +687,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // runs the other tile's work.  The V stage of item e is released after
         // PV(e,t1), which is issued while handling item e+1.
         struct Pending {
-          int valid, act1, f0, v_waited;
-        } pend = {0, 0, 0, 0};
+          int valid, act1, f0, v_waited, f1;  // f1: split mode only
+        } pend = {0, 0, 0, 0, 0};
         auto issue_pv = [&](int t, int flag) -> bool {
           if (!((pv_started >> t) & 1)) {
             if (!free_o(t)) return false;
@@ -695,7 +707,48 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_commit(&sm.pv_done[t]);
           return true;
         };
+        // Split mode: tile t's PV half by half as the softmax hands over P (flag:
+        // the halves any segment keeps, from the schedule), half 0's PV
+        // committed to pvh0 before half 1 is waited for.  The V stage must be in.
+        auto pv_split = [&](int t, int flag, int& v_waited) -> bool {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait_t(h == 0 ? &sm.p_full[t] : &sm.p_full1[t], (pph >> t) & 1u, wctx,
+                             pacc[2]))
+              return false;
+            if ((flag >> h) & 1) {
+              if (!v_waited) {
+                if (!mbar_wait_t(&sm.v_full[vs], vph, wctx, pacc[3])) return false;
+                v_waited = 1;
+              }
+              tc_fence_after();
+              if (!((pv_started >> t) & 1) && !free_o(t)) return false;
+              tc_fence_after();
+              const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * kKVTileBytes) >> 4);
+              uint32_t acc = (pv_started >> t) & 1;
+#pragma unroll
+              for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+                umma_ts(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + ((kk * 2048) >> 4),
+                        idesc_pv, acc);
+                acc = 1;
+              }
+              pv_started |= 1 << t;
+            }
+            umma_commit(h == 0 ? &sm.pvh0[t] : &sm.pv_done[t]);
+          }
+          pph ^= 1u << t;
+          return true;
+        };
         auto finish_prev = [&]() -> bool {
+          if (split_p) {
+            if (pend.act1 && !pv_split(1, pend.f1, pend.v_waited)) return false;
+            if (pend.f0 | pend.f1) {
+              umma_commit(&sm.v_empty[vs]);
+              if (++vs == kVStages) { vs = 0; vph ^= 1u; }
+            }
+            pend.valid = 0;
+            return true;
+          }
           int f1 = 0;
           if (pend.act1) {
             if (!mbar_wait_t(&sm.p_full[1], (pph >> 1) & 1u, wctx, pacc[2])) return false;
@@ -735,6 +788,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_commit(&sm.k_empty[ks]);
           if (++ks == kKStages) { ks = 0; kph ^= 1u; }
           int f0 = 0, v_waited = 0;
+          if (split_p) {
+            f0 = pf_tile_halves(mem, 0);
+            if ((act & 1) && !pv_split(0, f0, v_waited)) return false;
+            pend = {1, (act >> 1) & 1, f0, v_waited, pf_tile_halves(mem, 1)};
+            return true;
+          }
           if (act & 1) {
             if (!mbar_wait_t(&sm.p_full[0], pph & 1u, wctx, pacc[2])) return false;
             pph ^= 1u;
@@ -746,7 +805,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (!issue_pv(0, f0)) return false;
             }
           }
-          pend = {1, (act >> 1) & 1, f0, v_waited};
+          pend = {1, (act >> 1) & 1, f0, v_waited, 0};
           return true;
         };
         ok = pf_for_each<has_cols>(sc, gated ? pf_kb(sc) : &sc.bm[0][0], body);
@@ -930,6 +989,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // 2^8) from each half's max as it comes; if half 1 raises it, half 0's
         // P, already in TMEM, is scaled to the new m (rare after a row's first
         // tiles).  O and l of earlier tiles take the product of the factors.
+        // With split_p each half is handed over as soon as it is written, and
+        // O goes to the new scale before that half's P V is added.
         const int my_keep = segm;
         const int flag = tmask;
         float alpha = 1.f, psum = 0.f;
@@ -957,7 +1018,29 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
               }
             }
-            if (h == 1 && __any_sync(0xffffffffu, a_h != 1.f)) {
+            if (split_p) {
+              // half 0 was handed over already: O (earlier tiles, or for half 1
+              // also half 0's P V, once it has completed) goes to the new scale
+              // before this half's P V is added
+              if ((npv > 0 || h == 1) && __any_sync(0xffffffffu, a_h != 1.f)) {
+                if (h == 1) {
+                  pacc[4] += 1;
+                  if (!__all_sync(0xffffffffu,
+                                  mbar_wait_t(&sm.pvh0[t], pv_total & 1, wctx, pacc[1])))
+                    return false;
+                  tc_fence_after();
+                }
+                float ob[32];
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                  tmem_ld32(lane_addr + 128 + c * 32, ob);
+#pragma unroll
+                  for (int i = 0; i < 32; i += 2) mul2(ob[i], ob[i + 1], a_h);
+                  tmem_st32(lane_addr + 128 + c * 32, ob);
+                }
+              }
+              l *= a_h;
+            } else if (h == 1 && __any_sync(0xffffffffu, a_h != 1.f)) {
               pacc[4] += 1;
               tmem_wait_st();
               float pf[32];
@@ -985,13 +1068,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               add2(ps4[a], ps4[a + 1], p0, p1);
               pk[c >> 1] = pack_bf16x2(p0, p1);
             }
-            psum += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+            if (split_p) l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+            else psum += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
           } else {
 #pragma unroll
             for (int c = 0; c < 32; ++c) pk[c] = 0u;
           }
-          if (h == 0) tmem_st32_nowait(lane_addr, reinterpret_cast<const float*>(pk));
-          else tmem_st32(lane_addr + 32, reinterpret_cast<const float*>(pk));
+          if (split_p) {
+            tmem_st32(lane_addr + 32 * h, reinterpret_cast<const float*>(pk));
+            tc_fence_before();
+            mbar_arrive(h == 0 ? &sm.p_full[t] : &sm.p_full1[t]);
+          } else if (h == 0) {
+            tmem_st32_nowait(lane_addr, reinterpret_cast<const float*>(pk));
+          } else {
+            tmem_st32(lane_addr + 32, reinterpret_cast<const float*>(pk));
+          }
+        }
+        if (split_p) {  // l already took each half's factor and sum
+          ++npv;
+          ++pv_total;
+          return true;
         }
         // the commit behind s_full also covers the previous PV: O is stable here
         if (npv > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
