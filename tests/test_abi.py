@@ -105,6 +105,27 @@ def test_host_validation_rejects_before_launch(sb):
         sb.ERR_UNSUPPORTED
 
 
+def test_workspace_sizes(sb):
+    """The NSA workspace query is host arithmetic (no GPU): the workspace
+    holds the inverted index, the unit table and one fp32 accumulator row per
+    (token, head) with its sum and row-maximum key -- not one partial per
+    (token, head, slot).  Bad sizes give 0.  (The decode query sizes by the
+    device's SM count and needs a GPU.)"""
+    lib = ctypes.CDLL(sb.LIB_PATH)
+    lib.sbfa_varlen_selected_workspace_size.restype = ctypes.c_size_t
+    nsa = lib.sbfa_varlen_selected_workspace_size
+    total, H, topk = 98304, 4, 16
+    n = nsa(2, total, 65536, H, H, topk)
+    acc = total * H * 128 * 4
+    assert acc + 2 * total * H * 4 <= n < 0.26e9, n    # 0.23 GB on the bench workload
+    assert n < total * H * topk * 128 * 4 / 10          # far below per-slot fp32 partials
+    assert nsa(2, 2 * total, 65536, H, H, topk) > n
+    assert nsa(2, total, 65536, 2 * H, H, topk) > n
+    for bad in [(0, total, 65536, H, H, topk), (2, 0, 65536, H, H, topk),
+                (2, total, 65536, H, H, 0), (2, total, 0, H, H, topk)]:
+        assert nsa(*bad) == 0
+
+
 def test_package_fails_loudly_without_library(tmp_path, monkeypatch):
     import importlib.util
     import sys
