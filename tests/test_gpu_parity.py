@@ -584,6 +584,26 @@ def test_nsa_varlen_small_all_tokens(sb, seqlens):
     compare(o[None], lse[None], ro[None], rl[None], f"nsa small {seqlens}")
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (16, 1)])
+def test_nsa_varlen_gqa(sb, Hq, Hkv):
+    """Query heads sharing a kv head's selection (G = Hq / Hkv rows of a
+    unit per list entry): every token and head against the oracle."""
+    seqlens = (700, 300, 130)
+    rng = np.random.default_rng(70 + Hq)
+    total = sum(seqlens)
+    q = W.normal_bf16(rng, (total, Hq, 128))
+    k = W.normal_bf16(rng, (total, Hkv, 128))
+    v = W.normal_bf16(rng, (total, Hkv, 128))
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    sel = W.nsa_selection(np.random.default_rng(1070 + Hq), seqlens, Hkv, 64, 16)
+    st = sb.new_status("cuda")
+    o, lse = sb.fwd_varlen_selected(dev(q), dev(k), dev(v), torch.from_numpy(cu).cuda(),
+                                    max(seqlens), torch.from_numpy(sel).cuda(), status=st)
+    sb.check_status(st)
+    ro, rl = oracle.attend_selected_varlen(q, k, v, cu, sel, 64, True, W.default_scale())
+    compare(o[None], lse[None], ro[None], rl[None], f"nsa gqa Hq={Hq} Hkv={Hkv}")
+
+
 def test_nsa_varlen_large_key_space(sb):
     """max_seqlen far above the real lengths makes the (kv head, block) key
     space too large for the shared-memory histograms: the inverted index is
