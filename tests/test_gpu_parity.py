@@ -353,6 +353,24 @@ def test_gated_small_all_rows(sb):
     assert np.all(kept[0][:, np.triu_indices(n, 1)[0], np.triu_indices(n, 1)[1]] == 255)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2)])
+def test_gated_group_sizes(sb, Hq, Hkv):
+    """Unit shapes other than one GQA group of 4 at one q-block: G = 1 (four
+    consecutive q-blocks of one head, each segment with its own diagonal)
+    and G = 2 (two heads at two q-blocks).  Keep bits exact, all rows."""
+    wl, T = _gated_small(Hq=Hq, Hkv=Hkv, k_top=3)
+    q, k, v = dev(wl.q), dev(wl.k), dev(wl.v)
+    n = T.shape[1]
+    smax = torch.full((1, Hq, n, n), float("nan"), device="cuda")
+    keep = torch.full((1, Hq, n, n), 255, dtype=torch.uint8, device="cuda")
+    o, lse = sb.fwd_gated(q, k, v, torch.from_numpy(T).cuda(), smax_out=smax, keep_out=keep)
+    ro, rl, info = oracle.attend_gated(wl.q, wl.k, wl.v, T, 64, wl.scale, return_keep=True)
+    kept = keep.cpu().numpy()
+    flipped = _check_keep(info, smax.cpu().numpy(), kept, T, f"gated Hq={Hq} Hkv={Hkv}")
+    _regate(wl, kept, flipped, ro, rl)
+    compare(o, lse, ro, rl, f"gated Hq={Hq} Hkv={Hkv}")
+
+
 @pytest.mark.parametrize("L", [1000, 1090])
 def test_gated_ragged_length(sb, L):
     """A sequence length that is not a multiple of 64: the last q-block and
@@ -453,6 +471,24 @@ def test_vertical_slash_small(sb):
     ro, rl = oracle.attend_vertical_slash(wl.q, wl.k, wl.v, rbc, rbo, rcc, rci, 64, 64, True,
                                           wl.scale)
     compare(o, lse, ro, rl, "vs small")
+
+
+def test_vertical_slash_gqa(sb):
+    """Per-query-head lists over shared kv heads (Hq = 8, Hkv = 2): the
+    unit is one GQA group at one q-block, each segment with its own lists."""
+    wl = _vs_small(L=1536, H=8, nnz_v=96, nnz_s=120, seed=45)
+    L = wl.q.shape[1]
+    rng = np.random.default_rng(1045)
+    k = W.normal_bf16(rng, (1, L, 2, 128))
+    v = W.normal_bf16(rng, (1, L, 2, 128))
+    vert, slash = wl.meta["vertical"], wl.meta["slash"]
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    bc, bo, cc, ci = sb.convert_vertical_slash(sl, sl, torch.from_numpy(vert).cuda(),
+                                               torch.from_numpy(slash).cuda(), L)
+    o, lse = sb.fwd_vertical_slash(dev(wl.q), dev(k), dev(v), bc, bo, cc, ci, causal=True)
+    rbc, rbo, rcc, rci = oracle.convert_vertical_slash([L], [L], vert, slash, L, 64, 64, True)
+    ro, rl = oracle.attend_vertical_slash(wl.q, k, v, rbc, rbo, rcc, rci, 64, 64, True, wl.scale)
+    compare(o, lse, ro, rl, "vertical/slash gqa")
 
 
 def test_vertical_slash_columns_heavy(sb):
